@@ -1,0 +1,179 @@
+"""B200 (sm_100a) DeepSeek-V3 MoE layer forward pass: Python binding of the C ABI.
+
+Argument marshalling only: every step of the layer runs in the CUDA kernels
+of ``libmoe_b200.so`` (``include/moe.h``).  PyTorch supplies device memory and
+streams.  There is no CPU fallback: without the built library every call
+raises.
+
+    cfg = MoeConfig(d=7168, n_experts=256, n_groups=8, topk_groups=4, top_k=8,
+                    hidden=2048, n_shared=1, shared_hidden=2048, routed_scale=2.5)
+    ws = torch.empty(workspace_size(cfg, T), dtype=torch.uint8, device="cuda")
+    moe_forward(cfg, weights, x, bias, y, workspace=ws)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "moe.h")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_DEVICE, MOE_ERR_CUDA = range(6)
+MOE_F32, MOE_BF16, MOE_E4M3 = 0, 1, 2
+MOE_DEVERR_BAD_EXPERT, MOE_DEVERR_TIMEOUT, MOE_DEVERR_BAD_ROWS = 1, 2, 4
+
+_lib = None
+_lock = threading.Lock()
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}")
+
+
+class MoeConfig(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int), ("n_experts", ctypes.c_int), ("n_groups", ctypes.c_int),
+                ("topk_groups", ctypes.c_int), ("top_k", ctypes.c_int), ("hidden", ctypes.c_int),
+                ("n_shared", ctypes.c_int), ("shared_hidden", ctypes.c_int), ("routed_scale", ctypes.c_float),
+                ("act_dtype", ctypes.c_int), ("weight_dtype", ctypes.c_int)]
+
+    def __init__(self, d, n_experts, n_groups, topk_groups, top_k, hidden, n_shared=1, shared_hidden=None,
+                 routed_scale=2.5, act_dtype=MOE_BF16, weight_dtype=MOE_BF16):
+        super().__init__(d, n_experts, n_groups, topk_groups, top_k, hidden, n_shared,
+                         hidden if shared_hidden is None else shared_hidden, routed_scale, act_dtype, weight_dtype)
+
+
+class MoeWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "w_router", "w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down",
+        "ws_gate", "ws_up", "ws_down", "ss_gate", "ss_up", "ss_down")]
+
+
+def lib():
+    """The loaded ``libmoe_b200.so``; raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with fine_grained_moe_gemm_b200.build.build() "
+                                   "(there is no CPU fallback)")
+            L = ctypes.CDLL(LIB_PATH)
+            P, I = ctypes.c_void_p, ctypes.c_int
+            L.moe_workspace_size.restype = ctypes.c_size_t
+            L.moe_workspace_size.argtypes = [ctypes.POINTER(MoeConfig), I]
+            L.moe_route.restype = I
+            L.moe_route.argtypes = [ctypes.POINTER(MoeConfig), P, P, P, P, I, P, P, P]
+            L.moe_permute.restype = I
+            L.moe_permute.argtypes = [ctypes.POINTER(MoeConfig), P, I, P, P, P, P, P]
+            L.moe_forward.restype = I
+            L.moe_forward.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, I, P, I, I, P,
+                                      ctypes.c_size_t, P]
+            L.moe_device_error.restype = I
+            L.moe_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), P]
+            L.moe_status_string.restype = ctypes.c_char_p
+            L.moe_status_string.argtypes = [I]
+            L.moe_abi_version.restype = I
+            _lib = L
+    return _lib
+
+
+def declared_symbols() -> list[str]:
+    """Entry points declared in include/moe.h."""
+    text = open(HEADER_PATH).read()
+    return re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text)
+
+
+def status_string(status: int) -> str:
+    return lib().moe_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != MOE_OK:
+        raise MoeError(status, what)
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return MOE_F32
+    if t.dtype == torch.bfloat16:
+        return MOE_BF16
+    if t.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return MOE_E4M3
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _dev(t: torch.Tensor, name: str):
+    if t is not None and (not t.is_cuda or not t.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+def workspace_size(cfg: MoeConfig, T: int) -> int:
+    return int(lib().moe_workspace_size(ctypes.byref(cfg), int(T)))
+
+
+def moe_route(cfg: MoeConfig, x, w_router, logits, bias, topk_idx, topk_w, stream=None):
+    """Router + selection.  ``x=None``: ``logits`` is an input (logits-in mode)."""
+    for n, t in (("x", x), ("w_router", w_router), ("logits", logits), ("bias", bias), ("topk_idx", topk_idx),
+                 ("topk_w", topk_w)):
+        _dev(t, n)
+    T = logits.shape[0]
+    _check(lib().moe_route(ctypes.byref(cfg), _p(x), _p(w_router), _p(logits), _p(bias), T, _p(topk_idx),
+                           _p(topk_w), _stream(stream)), "moe_route")
+
+
+def moe_permute(cfg: MoeConfig, topk_idx, counts, offsets, src, inv, stream=None):
+    for n, t in (("topk_idx", topk_idx), ("counts", counts), ("offsets", offsets), ("src", src), ("inv", inv)):
+        _dev(t, n)
+    T = topk_idx.shape[0]
+    _check(lib().moe_permute(ctypes.byref(cfg), _p(topk_idx), T, _p(counts), _p(offsets), _p(src), _p(inv),
+                             _stream(stream)), "moe_permute")
+
+
+def make_weights(w: dict) -> MoeWeights:
+    """MoeWeights from a dict of CUDA tensors (keys as in ``MoeWeights``; missing keys are NULL)."""
+    mw = MoeWeights()
+    for name, _ in MoeWeights._fields_:
+        t = w.get(name)
+        if t is not None:
+            _dev(t, name)
+            setattr(mw, name, t.data_ptr())
+    return mw
+
+
+def moe_forward(cfg: MoeConfig, weights, x, bias, y, accumulate: bool = False, workspace=None, stream=None):
+    """y (+)= MoE(x).  ``weights`` is a MoeWeights or a dict of tensors; ``workspace`` a uint8 CUDA tensor of at
+    least ``workspace_size(cfg, T)`` bytes."""
+    for n, t in (("x", x), ("bias", bias), ("y", y), ("workspace", workspace)):
+        _dev(t, n)
+    mw = weights if isinstance(weights, MoeWeights) else make_weights(weights)
+    T = x.shape[0]
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().moe_forward(ctypes.byref(cfg), ctypes.byref(mw), _p(x), _p(bias), T, _p(y), _dtype_code(y),
+                             1 if accumulate else 0, _p(workspace), ws_bytes, _stream(stream)), "moe_forward")
+
+
+def device_error(stream=None) -> int:
+    """Reads and clears the device error word (synchronises the stream); returns the MOE_DEVERR_* bits."""
+    flags = ctypes.c_uint(0)
+    st = lib().moe_device_error(ctypes.byref(flags), _stream(stream))
+    if st not in (MOE_OK, MOE_ERR_DEVICE):
+        raise MoeError(st, "moe_device_error")
+    return int(flags.value)

@@ -1,0 +1,391 @@
+// C ABI of the MoE layer forward pass (include/moe.h): argument checks,
+// workspace layout, TMA tensor maps and the launch sequence.  Host code only.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/moe.h"
+#include "moe_launch.h"
+
+using namespace moe;
+
+namespace {
+
+// ------------------------------------------------------------------ checks
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status check_config(const moe_config* c) {
+    if (!c) return MOE_ERR_INVALID_ARG;
+    if (c->d <= 0 || c->d % 128 != 0) return MOE_ERR_INVALID_ARG;
+    if (c->n_experts <= 0 || c->n_experts > 1024) return MOE_ERR_INVALID_ARG;
+    if (c->n_groups <= 0 || c->n_groups > 32 || c->n_experts % c->n_groups != 0) return MOE_ERR_INVALID_ARG;
+    const int gs = c->n_experts / c->n_groups;
+    if (gs < 2) return MOE_ERR_INVALID_ARG;
+    if (c->topk_groups < 1 || c->topk_groups > c->n_groups) return MOE_ERR_INVALID_ARG;
+    if (c->top_k < 1 || c->top_k > 32 || c->top_k > c->topk_groups * gs) return MOE_ERR_INVALID_ARG;
+    if (c->hidden <= 0 || c->hidden % 128 != 0) return MOE_ERR_INVALID_ARG;
+    if (c->n_shared != 0 && c->n_shared != 1) return MOE_ERR_INVALID_ARG;
+    if (c->n_shared == 1 && (c->shared_hidden <= 0 || c->shared_hidden % 128 != 0)) return MOE_ERR_INVALID_ARG;
+    if (c->act_dtype != MOE_F32 && c->act_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (c->weight_dtype != MOE_BF16 && c->weight_dtype != MOE_E4M3) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+struct DevInfo {
+    int sm_count = 0;
+    int major = 0;
+};
+
+DevInfo dev_info() {
+    static std::mutex mu;
+    static DevInfo cache[64];
+    static bool have[64] = {};
+    int dev = 0;
+    DevInfo info;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return info;
+    std::lock_guard<std::mutex> g(mu);
+    if (dev < 64 && have[dev]) return cache[dev];
+    cudaDeviceGetAttribute(&info.sm_count, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&info.major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (dev < 64) {
+        cache[dev] = info;
+        have[dev] = true;
+    }
+    return info;
+}
+
+moe_status check_device(DevInfo* out) {
+    DevInfo i = dev_info();
+    if (i.major != 10 || i.sm_count <= 0) return MOE_ERR_UNSUPPORTED;
+    *out = i;
+    return MOE_OK;
+}
+
+// ------------------------------------------------------------------ TMA maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D row-major [rows, cols] map, box [box_rows, box_cols], 128-byte swizzle,
+// out-of-bounds elements read as zero.
+bool map_2d(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* ptr, uint64_t rows, uint64_t cols,
+            uint32_t box_rows, uint32_t box_cols) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool map_bf16(CUtensorMap* m, const void* p, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    return map_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p, rows, cols, box_rows, 64);
+}
+
+// ------------------------------------------------------------------ tiles
+// Token-chunk width of the grouped GEMMs from the expected rows per expert:
+// small chunks for decode (few tokens per expert), wide ones for prefill.
+int pick_bn(long long rows_per_expert) {
+    if (rows_per_expert <= 24) return 32;
+    if (rows_per_expert <= 48) return 64;
+    if (rows_per_expert <= 160) return 128;
+    return 256;
+}
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Workspace {
+    float* logits;
+    int32_t* idx;
+    float* w;
+    int32_t* counts;
+    int32_t* offsets;
+    int32_t* src;
+    int32_t* inv;
+    int32_t* row_tok;
+    float* row_coef;
+    int32_t* row_off;
+    int32_t* item_gu;
+    int32_t* item_dn;
+    __nv_bfloat16* x_perm;
+    __nv_bfloat16* h_perm;
+    float* y_acc;
+    size_t bytes;
+};
+
+// Lays out the workspace for T tokens from `base` (NULL: sizes only).
+Workspace layout(const moe_config* c, int T, void* base) {
+    Workspace w;
+    memset(&w, 0, sizeof(w));
+    const size_t E = c->n_experts, k = c->top_k, NG = E + c->n_shared;
+    const size_t rows = (size_t)T * k + (size_t)c->n_shared * T;
+    const size_t ldh = c->hidden > c->shared_hidden ? c->hidden : c->shared_hidden;
+    size_t off = 0;
+    uint8_t* b = static_cast<uint8_t*>(base);
+    auto take = [&](size_t bytes) -> void* {
+        void* p = base ? b + off : nullptr;
+        off = align_up(off + bytes, 1024);
+        return p;
+    };
+    w.logits = (float*)take((size_t)T * E * 4);
+    w.idx = (int32_t*)take((size_t)T * k * 4);
+    w.w = (float*)take((size_t)T * k * 4);
+    w.counts = (int32_t*)take(E * 4);
+    w.offsets = (int32_t*)take((E + 1) * 4);
+    w.src = (int32_t*)take((size_t)T * k * 4);
+    w.inv = (int32_t*)take((size_t)T * k * 4);
+    w.row_tok = (int32_t*)take(rows * 4);
+    w.row_coef = (float*)take(rows * 4);
+    w.row_off = (int32_t*)take((NG + 1) * 4);
+    w.item_gu = (int32_t*)take((NG + 1) * 4);
+    w.item_dn = (int32_t*)take((NG + 1) * 4);
+    w.x_perm = (__nv_bfloat16*)take(rows * (size_t)c->d * 2);
+    w.h_perm = (__nv_bfloat16*)take(rows * ldh * 2);
+    w.y_acc = (float*)take((size_t)T * c->d * 4);
+    w.bytes = off;
+    return w;
+}
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// Router logits on tensor cores (bf16 x) or CUDA cores (fp32 x), then selection.
+moe_status route_impl(const moe_config* c, const DevInfo& di, const void* x, const void* w_router, float* logits,
+                      const float* bias, int T, int32_t* idx, float* w, cudaStream_t s) {
+    if (x) {
+        if (c->act_dtype == MOE_F32) {
+            cudaError_t e = launch_router_f32(static_cast<const float*>(x),
+                                              static_cast<const __nv_bfloat16*>(w_router), T, c->d, c->n_experts,
+                                              logits, s);
+            if (e != cudaSuccess) return MOE_ERR_CUDA;
+        } else {
+            GemmArgs a;
+            memset(&a, 0, sizeof(a));
+            const int bn = T <= 256 ? 32 : 128;
+            if (!map_bf16(&a.a0, w_router, c->n_experts, c->d, 128)) return MOE_ERR_CUDA;
+            a.a1 = a.s0 = a.s1 = a.a0;
+            if (!map_bf16(&a.b, x, T, c->d, bn)) return MOE_ERR_CUDA;
+            a.item_off = nullptr;
+            a.n_rows_single = T;
+            a.K_routed = a.K_shared = c->d;
+            a.mt_routed = (c->n_experts + 127) / 128;
+            a.logits = logits;
+            a.n_logit_cols = c->n_experts;
+            const int items = a.mt_routed * ((T + bn - 1) / bn);
+            const int grid = items < di.sm_count ? items : di.sm_count;
+            if (launch_gemm(MODE_LOGITS, bn, &a, grid, s) != cudaSuccess) return MOE_ERR_CUDA;
+        }
+    }
+    return cuda_status(launch_select(logits, bias, T, c->n_experts, c->n_groups, c->topk_groups, c->top_k, idx, w, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+const char* moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+        case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+        case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    }
+    return "MOE_ERR_UNKNOWN";
+}
+
+size_t moe_workspace_size(const moe_config* cfg, int T_max) {
+    if (check_config(cfg) != MOE_OK || T_max < 0) return 0;
+    return layout(cfg, T_max, nullptr).bytes;
+}
+
+moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router, float* logits, const float* bias,
+                     int T, int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (T < 0) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!logits || !bias || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    if (x && (!w_router || !aligned16(x) || !aligned16(w_router))) return MOE_ERR_INVALID_ARG;
+    DevInfo di;
+    if ((st = check_device(&di)) != MOE_OK) return st;
+    return route_impl(cfg, di, x, w_router, logits, bias, T, topk_idx, topk_w, (cudaStream_t)stream);
+}
+
+moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, int T, int32_t* counts, int32_t* offsets,
+                       int32_t* src, int32_t* inv, moe_stream_t stream) {
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (T < 0) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!topk_idx || !counts || !offsets || !src || !inv) return MOE_ERR_INVALID_ARG;
+    DevInfo di;
+    if ((st = check_device(&di)) != MOE_OK) return st;
+    PermuteArgs a;
+    memset(&a, 0, sizeof(a));
+    a.idx = topk_idx;
+    a.T = T;
+    a.k = cfg->top_k;
+    a.E = cfg->n_experts;
+    a.counts = counts;
+    a.offsets = offsets;
+    a.src = src;
+    a.inv = inv;
+    return cuda_status(launch_permute(a, (cudaStream_t)stream));
+}
+
+moe_status moe_forward(const moe_config* cfg, const moe_weights* wt, const void* x, const float* bias, int T,
+                       void* y, moe_dtype y_dtype, int accumulate, void* workspace, size_t ws_bytes,
+                       moe_stream_t stream) {
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (T < 0 || (y_dtype != MOE_F32 && y_dtype != MOE_BF16) || (accumulate != 0 && accumulate != 1))
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!wt || !x || !bias || !y || !workspace) return MOE_ERR_INVALID_ARG;
+    if (!wt->w_router || !wt->w_gate || !wt->w_up || !wt->w_down) return MOE_ERR_INVALID_ARG;
+    if (cfg->n_shared && (!wt->ws_gate || !wt->ws_up || !wt->ws_down)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(wt->w_router) || !aligned16(wt->w_gate) ||
+        !aligned16(wt->w_up) || !aligned16(wt->w_down) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->n_shared && (!aligned16(wt->ws_gate) || !aligned16(wt->ws_up) || !aligned16(wt->ws_down)))
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->weight_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (ws_bytes < layout(cfg, T, nullptr).bytes) return MOE_ERR_WORKSPACE;
+    DevInfo di;
+    if ((st = check_device(&di)) != MOE_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+
+    const Workspace W = layout(cfg, T, workspace);
+    const int E = cfg->n_experts, k = cfg->top_k, d = cfg->d, H = cfg->hidden;
+    const int Hs = cfg->n_shared ? cfg->shared_hidden : H;
+    const int NG = E + cfg->n_shared;
+    const int rows_max = T * k + cfg->n_shared * T;
+    const int ldh = H > Hs ? H : Hs;
+    const int bn = pick_bn(((long long)T * k + E - 1) / E);
+
+    // (1)+(2) router and selection
+    st = route_impl(cfg, di, x, wt->w_router, W.logits, bias, T, W.idx, W.w, s);
+    if (st != MOE_OK) return st;
+
+    // (3) permutation + tile schedules
+    PermuteArgs pa;
+    memset(&pa, 0, sizeof(pa));
+    pa.idx = W.idx;
+    pa.T = T;
+    pa.k = k;
+    pa.E = E;
+    pa.counts = W.counts;
+    pa.offsets = W.offsets;
+    pa.src = W.src;
+    pa.inv = W.inv;
+    pa.topk_w = W.w;
+    pa.routed_scale = cfg->routed_scale;
+    pa.n_shared = cfg->n_shared;
+    pa.row_tok = W.row_tok;
+    pa.row_coef = W.row_coef;
+    pa.row_off = W.row_off;
+    pa.item_off_gu = W.item_gu;
+    pa.item_off_dn = W.item_dn;
+    pa.bn_gu = pa.bn_dn = bn;
+    pa.mt_gu_routed = H / 64;
+    pa.mt_gu_shared = Hs / 64;
+    pa.mt_dn = d / 128;
+    if (launch_permute(pa, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_gather(x, cfg->act_dtype == MOE_F32, d, W.row_tok, W.row_off + NG, rows_max, W.x_perm, di.sm_count,
+                      s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+
+    // (4) gate/up grouped GEMM with the SwiGLU epilogue -> h_perm
+    GemmArgs g;
+    memset(&g, 0, sizeof(g));
+    if (!map_bf16(&g.a0, wt->w_gate, (uint64_t)E * H, d, 64) || !map_bf16(&g.a1, wt->w_up, (uint64_t)E * H, d, 64))
+        return MOE_ERR_CUDA;
+    if (cfg->n_shared) {
+        if (!map_bf16(&g.s0, wt->ws_gate, Hs, d, 64) || !map_bf16(&g.s1, wt->ws_up, Hs, d, 64)) return MOE_ERR_CUDA;
+    } else {
+        g.s0 = g.a0;
+        g.s1 = g.a1;
+    }
+    if (!map_bf16(&g.b, W.x_perm, rows_max, d, bn)) return MOE_ERR_CUDA;
+    g.item_off = W.item_gu;
+    g.row_off = W.row_off;
+    g.n_groups = NG;
+    g.n_routed = E;
+    g.K_routed = g.K_shared = d;
+    g.mt_routed = H / 64;
+    g.mt_shared = Hs / 64;
+    g.rows_per_expert = H;
+    g.h = W.h_perm;
+    g.ldh = ldh;
+    if (launch_gemm(MODE_GATEUP, bn, &g, di.sm_count, s) != cudaSuccess) return MOE_ERR_CUDA;
+
+    // (5) down GEMM, routing-weight scale and un-permute scatter into fp32
+    float* yacc = y_dtype == MOE_F32 ? static_cast<float*>(y) : W.y_acc;
+    if ((y_dtype == MOE_BF16 || !accumulate) &&
+        cudaMemsetAsync(yacc, 0, (size_t)T * d * sizeof(float), s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    GemmArgs dn;
+    memset(&dn, 0, sizeof(dn));
+    if (!map_bf16(&dn.a0, wt->w_down, (uint64_t)E * d, H, 128)) return MOE_ERR_CUDA;
+    if (cfg->n_shared) {
+        if (!map_bf16(&dn.s0, wt->ws_down, d, Hs, 128)) return MOE_ERR_CUDA;
+    } else {
+        dn.s0 = dn.a0;
+    }
+    dn.a1 = dn.a0;
+    dn.s1 = dn.s0;
+    if (!map_bf16(&dn.b, W.h_perm, rows_max, ldh, bn)) return MOE_ERR_CUDA;
+    dn.item_off = W.item_dn;
+    dn.row_off = W.row_off;
+    dn.n_groups = NG;
+    dn.n_routed = E;
+    dn.K_routed = H;
+    dn.K_shared = Hs;
+    dn.mt_routed = dn.mt_shared = d / 128;
+    dn.rows_per_expert = d;
+    dn.y = yacc;
+    dn.row_coef = W.row_coef;
+    dn.row_tok = W.row_tok;
+    dn.ldy = d;
+    if (launch_gemm(MODE_DOWN, bn, &dn, di.sm_count, s) != cudaSuccess) return MOE_ERR_CUDA;
+
+    if (y_dtype == MOE_BF16 &&
+        launch_finalize_bf16(W.y_acc, static_cast<__nv_bfloat16*>(y), (size_t)T * d, accumulate != 0, s) !=
+            cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+moe_status moe_device_error(unsigned int* flags, moe_stream_t stream) {
+    if (!flags) return MOE_ERR_INVALID_ARG;
+    DevInfo di;
+    moe_status st = check_device(&di);
+    if (st != MOE_OK) return st;
+    if (read_clear_dev_error(flags, (cudaStream_t)stream) != cudaSuccess) return MOE_ERR_CUDA;
+    return *flags ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+}  // extern "C"

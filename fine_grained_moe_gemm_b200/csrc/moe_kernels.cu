@@ -1,0 +1,471 @@
+// Kernels of the MoE layer forward pass (sm_100a) and their launchers.
+//
+//   router_f32_kernel   fp32-activation router logits (CUDA cores)
+//   select_kernel       sigmoid, selection bias, group-limited top-k, weights
+//   permute_kernel      histogram / prefix sum / stable scatter by expert, and
+//                       the tile schedules of the grouped GEMMs
+//   gather_rows_kernel  x_perm = x[row_tok] (bf16)
+//   moe_gemm_kernel     tcgen05 grouped GEMM (moe_gemm.cuh)
+//   finalize_kernel     fp32 combine buffer -> bf16 output (+ residual)
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "moe_device.cuh"
+#include "moe_gemm.cuh"
+#include "moe_launch.h"
+
+namespace moe {
+
+// ============================================================================ router (fp32 x)
+// logits[t, e] = sum_c x[t, c] * Wr[e, c], fp32 products and fp32 sums
+// ("MoE router" box: gate(x.float())).  One block per token, one warp per
+// expert at a time, lanes stride over c, then a butterfly sum.
+__global__ void __launch_bounds__(256) router_f32_kernel(const float* __restrict__ x,
+                                                         const __nv_bfloat16* __restrict__ wr, int T, int d, int E,
+                                                         float* __restrict__ logits) {
+    const int t = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float* xr = x + (size_t)t * d;
+    for (int e = warp; e < E; e += 8) {
+        const __nv_bfloat16* w = wr + (size_t)e * d;
+        float acc = 0.0f;
+        for (int c = lane; c < d; c += 32) acc = fmaf(xr[c], __bfloat162float(w[c]), acc);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) logits[(size_t)t * E + e] = acc;
+    }
+}
+
+// ============================================================================ selection
+// Field guide cutaway 02 / "MoE router" box, one warp per token:
+//   s = sigmoid_spec(l); b = s + bias (selection only; -0 ranks as +0)
+//   group score = b(1) + b(2), the two strongest b of the group
+//   the topk_groups best groups are eligible
+//   slot j = the j-th best eligible expert by b
+//   w[j] = s[idx[j]] / S, S = sum of the selected s in ascending expert index
+// "a ranks before b": larger value, then lower index.
+__device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib) {
+    return va > vb || (va == vb && ia < ib);
+}
+
+__device__ __forceinline__ void warp_best(float& v, int& id) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        float ov = __shfl_xor_sync(0xffffffffu, v, o);
+        int oi = __shfl_xor_sync(0xffffffffu, id, o);
+        if (ranks_before(ov, oi, v, id)) {
+            v = ov;
+            id = oi;
+        }
+    }
+}
+
+constexpr int SELECT_WARPS = 8;
+
+__global__ void __launch_bounds__(SELECT_WARPS * 32) select_kernel(const float* __restrict__ logits,
+                                                                   const float* __restrict__ bias, int T, int E,
+                                                                   int G, int topk_groups, int k,
+                                                                   int32_t* __restrict__ idx_out,
+                                                                   float* __restrict__ w_out) {
+    extern __shared__ float ssm[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * SELECT_WARPS + warp;
+    if (t >= T) return;  // uniform per warp
+    float* s = ssm + (size_t)warp * 2 * E;
+    float* b = s + E;
+    const float* l = logits + (size_t)t * E;
+    for (int e = lane; e < E; e += 32) {
+        float sv = sigmoid_spec(l[e]);
+        float bv = __fadd_rn(sv, bias[e]);
+        if (bv == 0.0f) bv = 0.0f;
+        s[e] = sv;
+        b[e] = bv;
+    }
+    __syncwarp();
+    const int gs = E / G;
+    // group scores (lane g owns group g)
+    float gsc = -INFINITY;
+    if (lane < G) {
+        int i1 = -1, i2 = -1;
+        for (int e = lane * gs; e < (lane + 1) * gs; ++e) {
+            if (i1 < 0 || ranks_before(b[e], e, b[i1], i1)) {
+                i2 = i1;
+                i1 = e;
+            } else if (i2 < 0 || ranks_before(b[e], e, b[i2], i2)) {
+                i2 = e;
+            }
+        }
+        gsc = __fadd_rn(b[i1], b[i2]);
+        if (gsc == 0.0f) gsc = 0.0f;
+    }
+    unsigned gmask = 0;
+    for (int r = 0; r < topk_groups; ++r) {
+        bool cand = lane < G && !((gmask >> lane) & 1u);
+        float v = cand ? gsc : -INFINITY;
+        int id = cand ? lane : 0x7fffffff;
+        warp_best(v, id);
+        gmask |= 1u << id;
+    }
+    // experts: lane owns e = lane + 32 i
+    unsigned taken = 0;
+    int my_idx = -1;
+    for (int j = 0; j < k; ++j) {
+        float v = -INFINITY;
+        int id = 0x7fffffff;
+        for (int i = 0, e = lane; e < E; ++i, e += 32) {
+            if (((gmask >> (e / gs)) & 1u) && !((taken >> i) & 1u) && ranks_before(b[e], e, v, id)) {
+                v = b[e];
+                id = e;
+            }
+        }
+        warp_best(v, id);
+        if ((id & 31) == lane) taken |= 1u << (id >> 5);
+        if (lane == j) my_idx = id;
+    }
+    // S over the selected experts in ascending expert index
+    int rank = 0;
+    for (int jj = 0; jj < k; ++jj) {
+        int o = __shfl_sync(0xffffffffu, my_idx, jj);
+        if (lane < k && o < my_idx) ++rank;
+    }
+    const float my_s = lane < k ? s[my_idx] : 0.0f;
+    float S = 0.0f;
+    for (int r = 0; r < k; ++r) {
+        unsigned who = __ballot_sync(0xffffffffu, lane < k && rank == r);
+        float sv = __shfl_sync(0xffffffffu, my_s, __ffs(who) - 1);
+        S = __fadd_rn(S, sv);
+    }
+    if (lane < k) {
+        idx_out[(size_t)t * k + lane] = my_idx;
+        w_out[(size_t)t * k + lane] = __fdiv_rn(my_s, S);
+    }
+}
+
+// ============================================================================ permutation
+// "Routed experts" box (group all tokens per expert) as a counting sort:
+// histogram -> exclusive prefix sum -> stable scatter, one CTA of 1024 threads.
+// Stability (ascending t inside an expert) without a second sort: tokens are
+// processed in rounds of WR warps x 32 tokens; per warp and expert a 32-bit
+// mask of the lanes (tokens) that chose the expert gives the rank inside the
+// warp (popc of the lower lanes) and, prefix-summed over warps in order, the
+// warp's base.
+constexpr int PERM_THREADS = 1024;
+constexpr int PERM_SCAN_CAP = 2048;
+
+__device__ int block_excl_scan(int* a, int n, int* wsum) {
+    // in-place exclusive scan of a[0..n), n <= 2048, returns the total
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int v0 = 2 * tid < n ? a[2 * tid] : 0;
+    int v1 = 2 * tid + 1 < n ? a[2 * tid + 1] : 0;
+    int sum = v0 + v1;
+    int inc = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+    }
+    if (lane == 31) wsum[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        int w = wsum[lane];
+        int wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int y = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += y;
+        }
+        wsum[lane] = wi - w;  // exclusive
+        if (lane == 31) wsum[32] = wi;
+    }
+    __syncthreads();
+    int excl = wsum[warp] + inc - sum;
+    if (2 * tid < n) a[2 * tid] = excl;
+    if (2 * tid + 1 < n) a[2 * tid + 1] = excl + v0;
+    int total = wsum[32];
+    __syncthreads();
+    return total;
+}
+
+__global__ void __launch_bounds__(PERM_THREADS, 1) permute_kernel(PermuteArgs a, int WR) {
+    extern __shared__ int psm[];
+    const int E = a.E, T = a.T, k = a.k;
+    int* s_scan = psm;                              // [PERM_SCAN_CAP]
+    int* s_base = s_scan + PERM_SCAN_CAP;           // [E]
+    int* s_wsum = s_base + E;                       // [33] (+pad)
+    unsigned* s_mask = reinterpret_cast<unsigned*>(s_wsum + 64);  // [WR * E]
+    int* s_wbase = reinterpret_cast<int*>(s_mask + WR * E);       // [WR * E]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bool fwd = a.row_off != nullptr;
+    const int total_pairs = T * k;
+
+    for (int e = tid; e < E; e += PERM_THREADS) s_scan[e] = 0;
+    __syncthreads();
+    bool bad = false;
+    for (int p = tid; p < total_pairs; p += PERM_THREADS) {
+        int e = a.idx[p];
+        if (e >= 0 && e < E) atomicAdd(&s_scan[e], 1);
+        else bad = true;
+    }
+    if (bad) set_dev_error(MOE_DEVERR_BAD_EXPERT);
+    __syncthreads();
+    for (int e = tid; e < E; e += PERM_THREADS) a.counts[e] = s_scan[e];
+    __syncthreads();
+    int tot = block_excl_scan(s_scan, E, s_wsum);
+    for (int e = tid; e < E; e += PERM_THREADS) {
+        a.offsets[e] = s_scan[e];
+        s_base[e] = s_scan[e];
+    }
+    if (tid == 0) a.offsets[E] = tot;
+    __syncthreads();
+
+    if (fwd) {
+        const int NG = E + a.n_shared;
+        // group extents: routed experts back to back, the shared expert after them
+        for (int g = tid; g <= NG; g += PERM_THREADS)
+            a.row_off[g] = g <= E ? (g < E ? s_base[g] : tot) : tot + T;
+        __syncthreads();
+        for (int pass = 0; pass < 2; ++pass) {
+            const int bn = pass == 0 ? a.bn_gu : a.bn_dn;
+            for (int g = tid; g < NG; g += PERM_THREADS) {
+                int n = g < E ? a.counts[g] : T;
+                int mt = pass == 0 ? (g < E ? a.mt_gu_routed : a.mt_gu_shared) : a.mt_dn;
+                s_scan[g] = ((n + bn - 1) / bn) * mt;
+            }
+            __syncthreads();
+            int items = block_excl_scan(s_scan, NG, s_wsum);
+            int32_t* dst = pass == 0 ? a.item_off_gu : a.item_off_dn;
+            for (int g = tid; g < NG; g += PERM_THREADS) dst[g] = s_scan[g];
+            if (tid == 0) dst[NG] = items;
+            __syncthreads();
+        }
+        for (int t = tid; t < T * a.n_shared; t += PERM_THREADS) {
+            a.row_tok[tot + t] = t;
+            a.row_coef[tot + t] = 1.0f;
+        }
+    }
+
+    // stable scatter, rounds of WR warps x 32 tokens
+    const int TPR = WR * 32;
+    for (int base = 0; base < T; base += TPR) {
+        for (int i = tid; i < WR * E; i += PERM_THREADS) s_mask[i] = 0u;
+        __syncthreads();
+        const int t = base + warp * 32 + lane;
+        const bool mine = warp < WR && t < T;
+        if (mine) {
+            for (int j = 0; j < k; ++j) {
+                int e = a.idx[(size_t)t * k + j];
+                if (e >= 0 && e < E) atomicOr(&s_mask[warp * E + e], 1u << lane);
+            }
+        }
+        __syncthreads();
+        for (int e = tid; e < E; e += PERM_THREADS) {
+            int acc = s_base[e];
+            for (int w2 = 0; w2 < WR; ++w2) {
+                s_wbase[w2 * E + e] = acc;
+                acc += __popc(s_mask[w2 * E + e]);
+            }
+            s_base[e] = acc;
+        }
+        __syncthreads();
+        if (mine) {
+            const unsigned lower = (1u << lane) - 1u;
+            for (int j = 0; j < k; ++j) {
+                const int p = t * k + j;
+                int e = a.idx[p];
+                if (e >= 0 && e < E) {
+                    int row = s_wbase[warp * E + e] + __popc(s_mask[warp * E + e] & lower);
+                    a.src[row] = p;
+                    a.inv[p] = row;
+                    if (fwd) {
+                        a.row_tok[row] = t;
+                        a.row_coef[row] = a.routed_scale * a.topk_w[p];
+                    }
+                } else {
+                    a.inv[p] = -1;
+                }
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// ============================================================================ gather
+__global__ void __launch_bounds__(256) gather_rows_kernel(const void* __restrict__ x, int x_f32, int d,
+                                                          const int32_t* __restrict__ row_tok,
+                                                          const int32_t* __restrict__ n_rows_dev,
+                                                          __nv_bfloat16* __restrict__ xp) {
+    const int n_rows = *n_rows_dev;
+    const int nvec = d / 8;  // 8 bf16 per 16-byte vector
+    for (int r = blockIdx.x; r < n_rows; r += gridDim.x) {
+        const int t = row_tok[r];
+        uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)r * d);
+        if (x_f32) {
+            const float4* srcf = reinterpret_cast<const float4*>(static_cast<const float*>(x) + (size_t)t * d);
+            for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+                float4 a = srcf[2 * v], b = srcf[2 * v + 1];
+                __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y), p1 = __floats2bfloat162_rn(a.z, a.w);
+                __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y), p3 = __floats2bfloat162_rn(b.z, b.w);
+                dst[v] = make_uint4(*reinterpret_cast<uint32_t*>(&p0), *reinterpret_cast<uint32_t*>(&p1),
+                                    *reinterpret_cast<uint32_t*>(&p2), *reinterpret_cast<uint32_t*>(&p3));
+            }
+        } else {
+            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + (size_t)t * d);
+            for (int v = threadIdx.x; v < nvec; v += blockDim.x) dst[v] = src[v];
+        }
+    }
+}
+
+// ============================================================================ finalize
+__global__ void __launch_bounds__(256) finalize_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ y,
+                                                       size_t n8, int accumulate) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {
+        float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
+        float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+        float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        uint4* yp = reinterpret_cast<uint4*>(y) + i;
+        if (accumulate) {
+            uint4 old = *yp;
+            const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&old);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float2 f = __bfloat1622float2(o2[j]);
+                v[2 * j] += f.x;
+                v[2 * j + 1] += f.y;
+            }
+        }
+        uint32_t p[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+            p[j] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        *yp = make_uint4(p[0], p[1], p[2], p[3]);
+    }
+}
+
+// ============================================================================ launchers
+size_t gemm_args_size() { return sizeof(GemmArgs); }
+
+template <int MODE, int BN>
+static cudaError_t launch_gemm_t(const GemmArgs* args, int grid, cudaStream_t s) {
+    using C = GemmCfg<MODE, BN>;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(moe_gemm_kernel<MODE, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    moe_gemm_kernel<MODE, BN><<<grid, 192, C::SMEM_BYTES, s>>>(*args);
+    return cudaGetLastError();
+}
+
+template <int MODE>
+static int smem_t(int bn) {
+    switch (bn) {
+        case 32: return GemmCfg<MODE, 32>::SMEM_BYTES;
+        case 64: return GemmCfg<MODE, 64>::SMEM_BYTES;
+        case 128: return GemmCfg<MODE, 128>::SMEM_BYTES;
+        case 256: return GemmCfg<MODE, 256>::SMEM_BYTES;
+    }
+    return -1;
+}
+
+int gemm_smem_bytes(int mode, int bn) {
+    if (mode == MODE_GATEUP) return smem_t<GEMM_GATEUP>(bn);
+    if (mode == MODE_DOWN) return smem_t<GEMM_DOWN>(bn);
+    return smem_t<GEMM_LOGITS>(bn);
+}
+
+template <int MODE>
+static cudaError_t launch_mode(int bn, const GemmArgs* args, int grid, cudaStream_t s) {
+    switch (bn) {
+        case 32: return launch_gemm_t<MODE, 32>(args, grid, s);
+        case 64: return launch_gemm_t<MODE, 64>(args, grid, s);
+        case 128: return launch_gemm_t<MODE, 128>(args, grid, s);
+        case 256: return launch_gemm_t<MODE, 256>(args, grid, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_gemm(int mode, int bn, const GemmArgs* args, int grid, cudaStream_t s) {
+    if (mode == MODE_GATEUP) return launch_mode<GEMM_GATEUP>(bn, args, grid, s);
+    if (mode == MODE_DOWN) return launch_mode<GEMM_DOWN>(bn, args, grid, s);
+    return launch_mode<GEMM_LOGITS>(bn, args, grid, s);
+}
+
+cudaError_t launch_router_f32(const float* x, const __nv_bfloat16* wr, int T, int d, int E, float* logits,
+                              cudaStream_t s) {
+    router_f32_kernel<<<T, 256, 0, s>>>(x, wr, T, d, E, logits);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_select(const float* logits, const float* bias, int T, int E, int G, int tg, int k, int32_t* idx,
+                          float* w, cudaStream_t s) {
+    const int blocks = (T + SELECT_WARPS - 1) / SELECT_WARPS;
+    const size_t smem = (size_t)SELECT_WARPS * 2 * E * sizeof(float);
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             SELECT_WARPS * 2 * 1024 * (int)sizeof(float));
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    select_kernel<<<blocks, SELECT_WARPS * 32, smem, s>>>(logits, bias, T, E, G, tg, k, idx, w);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s) {
+    int WR = 8192 / a.E;
+    WR = WR > 32 ? 32 : (WR < 1 ? 1 : WR);
+    const size_t smem = (size_t)(PERM_SCAN_CAP + a.E + 64) * 4 + (size_t)2 * WR * a.E * 4;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    permute_kernel<<<1, PERM_THREADS, smem, s>>>(a, WR);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const void* x, bool x_f32, int d, const int32_t* row_tok, const int32_t* n_rows_dev,
+                          int max_rows, __nv_bfloat16* x_perm, int n_sm, cudaStream_t s) {
+    int grid = max_rows < n_sm * 8 ? max_rows : n_sm * 8;
+    if (grid < 1) grid = 1;
+    gather_rows_kernel<<<grid, 256, 0, s>>>(x, x_f32 ? 1 : 0, d, row_tok, n_rows_dev, x_perm);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_finalize_bf16(const float* acc, __nv_bfloat16* y, size_t n, bool accumulate, cudaStream_t s) {
+    size_t n8 = n / 8;
+    size_t grid = (n8 + 255) / 256;
+    if (grid > 148 * 16) grid = 148 * 16;
+    if (grid < 1) grid = 1;
+    finalize_kernel<<<(unsigned)grid, 256, 0, s>>>(acc, y, n8, accumulate ? 1 : 0);
+    return cudaGetLastError();
+}
+
+cudaError_t read_clear_dev_error(unsigned int* flags, cudaStream_t s) {
+    unsigned int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(flags, g_dev_error, sizeof(unsigned int), 0,
+                                              cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return e;
+    e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return e;
+    return cudaMemcpyToSymbolAsync(g_dev_error, &zero, sizeof(unsigned int), 0, cudaMemcpyHostToDevice, s) ==
+                   cudaSuccess
+               ? cudaStreamSynchronize(s)
+               : cudaGetLastError();
+}
+
+}  // namespace moe

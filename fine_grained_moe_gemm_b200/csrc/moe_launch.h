@@ -1,0 +1,76 @@
+// Host-side launch interface between the C ABI (moe_api.cu) and the kernels
+// (moe_kernels.cu).  Internal; not installed.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Arguments of the grouped GEMM kernel (moe_gemm.cuh), passed by value.
+struct GemmArgs {
+    CUtensorMap a0;  // routed A: GATEUP W_gate [E*H, d] (box 64x64) | DOWN W_down [E*d, H] (box 128x64) | LOGITS Wr [E, d]
+    CUtensorMap a1;  // GATEUP: W_up [E*H, d] (box 64x64)
+    CUtensorMap s0;  // shared A: GATEUP Ws_gate [Hs, d] | DOWN Ws_down [d, Hs]
+    CUtensorMap s1;  // GATEUP: Ws_up [Hs, d]
+    CUtensorMap b;   // B rows: x_perm [rows, d] | h_perm [rows, ldh] | x [T, d]; box BN x 64
+    const int* item_off;   // [n_groups + 1] prefix of work items per group; NULL: one group of n_rows_single rows
+    const int* row_off;    // [n_groups + 1] first B row of each group
+    int n_groups;
+    int n_routed;          // groups >= n_routed are the shared expert
+    int n_rows_single;
+    int K_routed, K_shared;
+    int mt_routed, mt_shared;  // M tiles per group
+    int rows_per_expert;       // A rows per routed expert (H for GATEUP, d for DOWN)
+    __nv_bfloat16* h;          // GATEUP output
+    int ldh;
+    float* y;                  // DOWN output (fp32, accumulated)
+    const float* row_coef;
+    const int* row_tok;
+    int ldy;
+    float* logits;             // LOGITS output
+    int n_logit_cols;
+};
+
+enum { MODE_GATEUP = 0, MODE_DOWN = 1, MODE_LOGITS = 2 };
+
+struct PermuteArgs {
+    const int32_t* idx;
+    int T, k, E;
+    int32_t* counts;   // [E]
+    int32_t* offsets;  // [E + 1]
+    int32_t* src;      // [T * k]
+    int32_t* inv;      // [T * k]
+    // forward mode (row_off != nullptr): per-row token / coefficient tables and
+    // the tile schedules of the two grouped GEMMs
+    const float* topk_w;
+    float routed_scale;
+    int n_shared;
+    int32_t* row_tok;      // [T * k + n_shared * T]
+    float* row_coef;       // [T * k + n_shared * T]
+    int32_t* row_off;      // [E + n_shared + 1]
+    int32_t* item_off_gu;  // [E + n_shared + 1]
+    int32_t* item_off_dn;  // [E + n_shared + 1]
+    int bn_gu, bn_dn;
+    int mt_gu_routed, mt_gu_shared, mt_dn;
+};
+
+size_t gemm_args_size();
+int gemm_smem_bytes(int mode, int bn);
+// grid: persistent CTAs (one per SM at most).
+cudaError_t launch_gemm(int mode, int bn, const GemmArgs* args, int grid, cudaStream_t s);
+cudaError_t launch_router_f32(const float* x, const __nv_bfloat16* wr, int T, int d, int E, float* logits,
+                              cudaStream_t s);
+cudaError_t launch_select(const float* logits, const float* bias, int T, int E, int G, int tg, int k,
+                          int32_t* idx, float* w, cudaStream_t s);
+cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
+// x_perm[r, :] = x[row_tok[r], :] (fp32 input rounded to bf16) for r < row_off[n_groups]
+cudaError_t launch_gather(const void* x, bool x_f32, int d, const int32_t* row_tok, const int32_t* n_rows_dev,
+                          int max_rows, __nv_bfloat16* x_perm, int n_sm, cudaStream_t s);
+// y[i] = bf16(acc[i] (+ y[i]))
+cudaError_t launch_finalize_bf16(const float* acc, __nv_bfloat16* y, size_t n, bool accumulate, cudaStream_t s);
+cudaError_t read_clear_dev_error(unsigned int* flags, cudaStream_t s);
+
+}  // namespace moe

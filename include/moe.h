@@ -1,0 +1,177 @@
+/*
+ * moe.h - C ABI of the B200 (sm_100a) DeepSeek-V3 MoE layer forward pass.
+ *
+ * The layer, as the pages define it:
+ *   - "DeepSeek-V3" (ainfra.dev llm-vis): "Mixture-of-Experts FFN" box (forward:
+ *     router, routed experts, shared expert), "MoE router" box (sigmoid scores,
+ *     selection-only bias, renormalised weights, routed scaling x2.5, router in
+ *     fp32), "Routed experts" box (grouped dispatch of all tokens per expert),
+ *     "Shared expert" box, "Expert combine" box
+ *     (y = 2.5 * sum_i w_i e_i(x) + shared(x)), "SwiGLU MLP" box
+ *     (W_down(SiLU(W_gate x) * W_up x)), "Residual add" box.
+ *   - "DeepSeek V3" field guide (curiouscaliboi), cutaway 02 "Fine-grained expert
+ *     routing": 8 groups of 32, each scored by its two strongest bias-adjusted
+ *     expert scores, top 4 groups eligible, top 8 experts inside them, weights
+ *     from the unbiased sigmoid renormalised to one, no token dropped.
+ *   - "Teardown: DeepSeek-V3", section 6 (sizes, bias for selection only) and
+ *     section 10 (FP8: E4M3, 1x128 activation tiles, 128x128 weight blocks,
+ *     router in higher precision).
+ *
+ * Conventions shared by every entry point
+ *   - All array arguments are DEVICE pointers (cudaMalloc'd or torch tensors'
+ *     data_ptr), row-major and densely packed, owned by the caller.  The
+ *     library allocates no device memory per call and keeps no per-call state.
+ *     Tensor-operand pointers (x, weights, workspace) must be 16-byte aligned.
+ *   - Every call is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and returns without synchronising the host.
+ *   - Errors found on the host (bad sizes, NULL or misaligned pointers) return
+ *     MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED before anything is enqueued.
+ *     A failed launch returns MOE_ERR_CUDA.  Errors found on the device (an
+ *     expert id out of range, a pipeline wait that ran past its time limit) set
+ *     bits in a per-device error word that moe_device_error() reads; kernels
+ *     never trap.
+ *   - T = 0 is valid and enqueues nothing.
+ *   - Requires an sm_100 device (B200); other devices get MOE_ERR_UNSUPPORTED.
+ */
+#ifndef MOE_B200_MOE_H
+#define MOE_B200_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef struct CUstream_st* moe_stream_t;   /* same type as cudaStream_t */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,   /* NULL / misaligned pointer, inconsistent sizes */
+    MOE_ERR_UNSUPPORTED = 2,   /* valid but not implemented (dtype combination, device) */
+    MOE_ERR_WORKSPACE = 3,     /* workspace smaller than moe_workspace_size() */
+    MOE_ERR_DEVICE = 4,        /* the device error word is non-zero */
+    MOE_ERR_CUDA = 5           /* a CUDA runtime call or launch failed */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_E4M3 = 2 } moe_dtype;
+
+/* Device error word bits (moe_device_error). */
+#define MOE_DEVERR_BAD_EXPERT 0x1u    /* a routed expert id outside [0, n_experts) */
+#define MOE_DEVERR_TIMEOUT    0x2u    /* a pipeline wait exceeded its limit */
+#define MOE_DEVERR_BAD_ROWS   0x4u    /* a tile schedule entry outside its buffer */
+
+/* Layer shape ("Teardown: DeepSeek-V3", At a glance + section 6; field guide
+ * cutaway 02).  Constraints checked by every entry point:
+ *   d % 128 == 0, hidden % 128 == 0, shared_hidden % 128 == 0 (0 if n_shared = 0),
+ *   n_experts <= 1024, n_experts % n_groups == 0, group size >= 2, n_groups <= 32,
+ *   1 <= topk_groups <= n_groups, 1 <= top_k <= min(32, topk_groups * group size),
+ *   n_shared in {0, 1}, act_dtype in {F32, BF16}, weight_dtype in {BF16, E4M3}. */
+typedef struct {
+    int d;               /* model width (7168) */
+    int n_experts;       /* routed experts E (256) */
+    int n_groups;        /* expert groups G (8) */
+    int topk_groups;     /* eligible groups per token (4) */
+    int top_k;           /* routed experts per token k (8) */
+    int hidden;          /* routed expert SwiGLU width H (2048) */
+    int n_shared;        /* shared experts, 0 or 1 (1) */
+    int shared_hidden;   /* shared expert width Hs (2048) */
+    float routed_scale;  /* routed scaling factor (2.5) */
+    moe_dtype act_dtype;     /* x: MOE_F32 or MOE_BF16 */
+    moe_dtype weight_dtype;  /* routed + shared expert weights: MOE_BF16 or MOE_E4M3 */
+} moe_config;
+
+/* Layer weights, nn.Linear layout ([out, in], K contiguous), experts stacked.
+ * The router weight is always bf16 (the router stays in high precision).
+ * E4M3 expert weights come with one fp32 scale per 128x128 block. */
+typedef struct {
+    const void* w_router;   /* [E, d] bf16 */
+    const void* w_gate;     /* [E, H, d] bf16 | e4m3 */
+    const void* w_up;       /* [E, H, d] bf16 | e4m3 */
+    const void* w_down;     /* [E, d, H] bf16 | e4m3 */
+    const float* s_gate;    /* e4m3 only: [E, H/128, d/128] */
+    const float* s_up;      /* e4m3 only: [E, H/128, d/128] */
+    const float* s_down;    /* e4m3 only: [E, d/128, H/128] */
+    const void* ws_gate;    /* shared expert [Hs, d] */
+    const void* ws_up;      /* shared expert [Hs, d] */
+    const void* ws_down;    /* shared expert [d, Hs] */
+    const float* ss_gate;   /* e4m3 only: [Hs/128, d/128] */
+    const float* ss_up;     /* e4m3 only: [Hs/128, d/128] */
+    const float* ss_down;   /* e4m3 only: [d/128, Hs/128] */
+} moe_weights;
+
+/* Bytes of device workspace moe_forward needs for up to T_max tokens
+ * (0 on invalid config).  The workspace holds the router logits, the routing,
+ * the permutation, the tile schedule, the permuted activations, the SwiGLU
+ * output h and the fp32 combine buffer. */
+MOE_API size_t moe_workspace_size(const moe_config* cfg, int T_max);
+
+/* Stages 1+2: router and selection ("MoE router" box; field guide cutaway 02).
+ *   x != NULL: logits[T,E] (fp32, written) = x[T,d] . w_router[E,d]^T with fp32
+ *              accumulation; x is cfg->act_dtype (fp32 or bf16).
+ *   x == NULL: logits[T,E] is an input (logits-in mode).
+ * Then s = sigmoid(logits); b = s + bias (selection only); group score = sum of
+ * the two largest b in the group; the topk_groups best groups are eligible;
+ * topk_idx[T,k] (int32) = the k best experts by b among them, in descending b
+ * (ties: lower index first); topk_w[T,k] (fp32) = s[idx] / sum of the selected
+ * s taken in ascending expert index, so the weights sum to 1 and are NOT
+ * multiplied by routed_scale.  The sigmoid is a fixed fp32 formula (Cody-Waite
+ * reduction and a degree-7 Taylor polynomial, correctly rounded operations
+ * only), so identical logits give bit-identical idx and w on any device.
+ * bias: [E] fp32.  Logits must be finite. */
+MOE_API moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router, float* logits,
+                     const float* bias, int T, int32_t* topk_idx, float* topk_w, moe_stream_t stream);
+
+/* Stage 3: permutation ("Routed experts" box: group all tokens per expert).
+ * Counting sort of the T*k (token, slot) pairs by expert, ascending token
+ * inside each expert (the order is unique: a token picks an expert once).
+ *   counts[E]    number of pairs per expert
+ *   offsets[E+1] exclusive prefix sum of counts; offsets[E] = T*k
+ *   src[T*k]     src[row] = t*k + j for the pair in permuted position row
+ *   inv[T*k]     inv[t*k + j] = row
+ * An id outside [0, E) sets MOE_DEVERR_BAD_EXPERT and is skipped. */
+MOE_API moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, int T, int32_t* counts,
+                       int32_t* offsets, int32_t* src, int32_t* inv, moe_stream_t stream);
+
+/* Stages 1-5: the whole layer ("Mixture-of-Experts FFN" forward; "Expert
+ * combine" box; "Residual add" box):
+ *   y[t] (+)= routed_scale * sum_j w[t,j] * expert_{idx[t,j]}(x[t]) + shared(x[t])
+ * expert(x) = W_down (SiLU(W_gate x) * (W_up x)), SiLU(z) = z * sigmoid(z).
+ * x: [T, d] cfg->act_dtype (fp32 input is rounded to bf16 for the experts; with
+ * E4M3 weights it is quantised to e4m3 per token and 128-channel block).
+ * y: [T, d] in y_dtype (MOE_F32 or MOE_BF16); accumulate = 0 overwrites y,
+ * accumulate = 1 adds the layer output to y (the residual stream).
+ * The expert GEMMs run on tcgen05 tensor cores with fp32 accumulation; h is
+ * stored in bf16 (e4m3 with 1x128 scales for E4M3 weights).  The combine adds
+ * fp32 partial sums with atomics, so the summation order of a token's 9
+ * expert outputs may vary between runs (within fp32 rounding).
+ * workspace: device buffer of ws_bytes >= moe_workspace_size(cfg, T),
+ * 256-byte aligned; it is overwritten. */
+MOE_API moe_status moe_forward(const moe_config* cfg, const moe_weights* w, const void* x, const float* bias,
+                       int T, void* y, moe_dtype y_dtype, int accumulate, void* workspace,
+                       size_t ws_bytes, moe_stream_t stream);
+
+/* Reads and clears the calling thread's current device's error word.  This
+ * call synchronises `stream` (it waits for the work enqueued before it).
+ * *flags receives the MOE_DEVERR_* bits; returns MOE_ERR_DEVICE if any is set. */
+MOE_API moe_status moe_device_error(unsigned int* flags, moe_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+MOE_API const char* moe_status_string(moe_status s);
+
+/* MOE_ABI_VERSION of the loaded library. */
+MOE_API int moe_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_MOE_H */

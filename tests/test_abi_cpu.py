@@ -1,0 +1,103 @@
+"""The C ABI library on the host (no GPU needed): it loads, exports every
+entry point include/moe.h declares, and rejects invalid arguments before it
+touches a device."""
+import ctypes
+
+import pytest
+
+import fine_grained_moe_gemm_b200 as moe
+from fine_grained_moe_gemm_b200 import build as moe_build
+from moe_testlib import cfg_of
+from workloads import WORKLOADS
+
+
+@pytest.fixture(scope="module")
+def L():
+    moe_build.build()
+    return moe.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = moe.declared_symbols()
+    assert set(names) >= {"moe_route", "moe_permute", "moe_forward", "moe_workspace_size", "moe_device_error",
+                          "moe_status_string", "moe_abi_version"}
+    for n in names:
+        assert hasattr(L, n), n
+    assert L.moe_abi_version() == 1
+
+
+def test_status_strings(L):
+    assert moe.status_string(moe.MOE_OK) == "MOE_OK"
+    assert moe.status_string(moe.MOE_ERR_WORKSPACE) == "MOE_ERR_WORKSPACE"
+    assert moe.status_string(99) == "MOE_ERR_UNKNOWN"
+
+
+def test_workspace_size(L):
+    cfg = cfg_of(WORKLOADS["decode"])
+    assert moe.workspace_size(cfg, 0) > 0
+    s128, s4096 = moe.workspace_size(cfg, 128), moe.workspace_size(cfg, 4096)
+    assert s4096 > s128
+    # dominated by the permuted activations (9T x d bf16), h (9T x H bf16) and the fp32 combine buffer
+    T = 4096
+    core = 9 * T * 7168 * 2 + 9 * T * 2048 * 2 + T * 7168 * 4
+    assert core <= s4096 <= core * 1.05
+    bad = cfg_of(WORKLOADS["decode"])
+    bad.n_groups = 7
+    assert moe.workspace_size(bad, 128) == 0
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("d", 100, moe.MOE_ERR_INVALID_ARG),           # not a multiple of 128
+    ("n_groups", 7, moe.MOE_ERR_INVALID_ARG),      # 256 % 7 != 0
+    ("topk_groups", 9, moe.MOE_ERR_INVALID_ARG),
+    ("top_k", 0, moe.MOE_ERR_INVALID_ARG),
+    ("hidden", 1000, moe.MOE_ERR_INVALID_ARG),
+    ("n_shared", 2, moe.MOE_ERR_INVALID_ARG),
+    ("act_dtype", moe.MOE_E4M3, moe.MOE_ERR_UNSUPPORTED),
+])
+def test_invalid_config_rejected_before_device(L, field, value, status):
+    cfg = cfg_of(WORKLOADS["decode"])
+    setattr(cfg, field, value)
+    P = ctypes.c_void_p
+    st = L.moe_route(ctypes.byref(cfg), None, None, P(16), P(16), 4, P(16), P(16), None)
+    assert st == status
+    st = L.moe_permute(ctypes.byref(cfg), P(16), 4, P(16), P(16), P(16), P(16), None)
+    assert st == status
+    w = moe.MoeWeights()
+    st = L.moe_forward(ctypes.byref(cfg), ctypes.byref(w), P(16), P(16), 4, P(16), moe.MOE_BF16, 0, P(1024),
+                       1 << 30, None)
+    assert st == status
+
+
+def test_null_and_negative_arguments(L):
+    cfg = cfg_of(WORKLOADS["decode"])
+    P = ctypes.c_void_p
+    assert L.moe_route(ctypes.byref(cfg), None, None, None, P(16), 4, P(16), P(16), None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_route(ctypes.byref(cfg), None, None, P(16), P(16), -1, P(16), P(16), None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_permute(ctypes.byref(cfg), None, 4, P(16), P(16), P(16), P(16), None) == moe.MOE_ERR_INVALID_ARG
+    # T = 0 is a valid no-op even without a device
+    assert L.moe_permute(ctypes.byref(cfg), None, 0, None, None, None, None, None) == moe.MOE_OK
+    w = moe.MoeWeights(w_router=16, w_gate=16, w_up=16, w_down=16, ws_gate=16, ws_up=16, ws_down=16)
+    # misaligned x
+    assert L.moe_forward(ctypes.byref(cfg), ctypes.byref(w), P(18), P(16), 4, P(16), moe.MOE_BF16, 0, P(1024),
+                         1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+    # workspace too small
+    assert L.moe_forward(ctypes.byref(cfg), ctypes.byref(w), P(16), P(16), 4, P(16), moe.MOE_BF16, 0, P(1024),
+                         1024, None) == moe.MOE_ERR_WORKSPACE
+    # bad output dtype / accumulate flag
+    assert L.moe_forward(ctypes.byref(cfg), ctypes.byref(w), P(16), P(16), 4, P(16), moe.MOE_E4M3, 0, P(1024),
+                         1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_forward(ctypes.byref(cfg), ctypes.byref(w), P(16), P(16), 4, P(16), moe.MOE_BF16, 2, P(1024),
+                         1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_no_device_means_unsupported_not_fallback(L):
+    """Valid arguments on a machine without an sm_100 device: the library refuses
+    (there is no CPU fallback).  On a B200 this test is skipped."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    cfg = cfg_of(WORKLOADS["decode"])
+    P = ctypes.c_void_p
+    st = L.moe_permute(ctypes.byref(cfg), P(16), 4, P(16), P(16), P(16), P(16), None)
+    assert st == moe.MOE_ERR_UNSUPPORTED

@@ -1,0 +1,136 @@
+"""GPU parity of the whole layer (moe_forward through the C ABI) against the oracle.
+
+Tolerance (the layer-output bar): max |err| <= 1e-2 x RMS(y_ref) for the fp32
+output against the oracle's unrounded fp64 output; the bf16 output adds one
+bf16 ulp of |y_ref| for its own storage rounding.  The oracle consumes the
+GPU's router logits (checked separately within tolerance) so that both sides
+route identically; the routing itself is compared bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import fine_grained_moe_gemm_b200 as moe
+from moe_testlib import assert_close_bf16, assert_close_rms, cfg_of, oracle_layer, weights_for_forward, x_host
+from workloads import WORKLOADS, make_inputs, make_residual, make_x
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+REL = 1e-2
+
+_cache = {}
+
+
+def inputs(name, device_gen):
+    """Full-size inputs are generated once per workload on the GPU (weights do not depend on T)."""
+    key = (name, device_gen)
+    if key not in _cache:
+        _cache.clear()
+        torch.cuda.empty_cache()
+        wl = WORKLOADS[name]
+        W = make_inputs(wl, device_gen)
+        _cache[key] = {k: v.to(DEV) for k, v in W.items()}
+    return _cache[key]
+
+
+def run_forward(wl, W, x, y_dtype=torch.float32, accumulate=False, y0=None):
+    cfg = cfg_of(wl)
+    T = x.shape[0]
+    ws = torch.empty(moe.workspace_size(cfg, T), dtype=torch.uint8, device=DEV)
+    y = y0.clone() if y0 is not None else torch.empty((T, wl.d), dtype=y_dtype, device=DEV)
+    moe.moe_forward(cfg, weights_for_forward(W), x, W["bias"], y, accumulate=accumulate, workspace=ws)
+    torch.cuda.synchronize()
+    assert moe.device_error() == 0
+    return y
+
+
+def gpu_routing(wl, W, x):
+    cfg = cfg_of(wl)
+    T = x.shape[0]
+    logits = torch.empty((T, wl.n_experts), dtype=torch.float32, device=DEV)
+    idx = torch.empty((T, wl.top_k), dtype=torch.int32, device=DEV)
+    w = torch.empty((T, wl.top_k), dtype=torch.float32, device=DEV)
+    moe.moe_route(cfg, x, W["w_router"], logits, W["bias"], idx, w)
+    torch.cuda.synchronize()
+    l = logits.cpu().numpy()
+    ridx, rw = oracle.select(l, W["bias"].cpu().numpy(), wl.n_groups, wl.topk_groups, wl.top_k)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    assert np.array_equal(w.cpu().numpy().view(np.uint32), rw.view(np.uint32))
+    return ridx, rw
+
+
+def oracle_y(wl, W, x, tokens):
+    idx, w = gpu_routing(wl, W, x)
+    need = np.unique(idx[tokens])
+    L = oracle_layer(wl, W, need)
+    return oracle.expert_tokens(L, x_host(x), idx, w, tokens)
+
+
+# ----------------------------------------------------------------------------- tiny workload (full check)
+
+@pytest.mark.parametrize("T", [64, 1, 2, 3, 127, 129, 600])
+def test_tiny_full(T):
+    wl = WORKLOADS["tiny"]
+    W = inputs("tiny", "cpu")
+    x = make_x(wl, "cpu", T=T).to(DEV)
+    ref = oracle_y(wl, W, x, np.arange(T))
+    y = run_forward(wl, W, x, torch.float32)
+    assert_close_rms(y.cpu().numpy(), ref, REL)
+    yb = run_forward(wl, W, x, torch.bfloat16)
+    assert_close_bf16(yb, ref, REL)
+
+
+def test_tiny_accumulate_into_residual():
+    wl = WORKLOADS["tiny"]
+    W = inputs("tiny", "cpu")
+    x = make_x(wl, "cpu").to(DEV)
+    ref = oracle_y(wl, W, x, np.arange(wl.T))
+    r32 = make_residual(wl, "cpu", dtype=torch.float32).to(DEV)
+    y = run_forward(wl, W, x, accumulate=True, y0=r32)
+    assert_close_rms(y.cpu().numpy(), ref + r32.cpu().numpy().astype(np.float64), REL)
+    rb = make_residual(wl, "cpu", dtype=torch.bfloat16).to(DEV)
+    yb = run_forward(wl, W, x, accumulate=True, y0=rb)
+    assert_close_bf16(yb, ref + rb.float().cpu().numpy().astype(np.float64), REL)
+
+
+# ----------------------------------------------------------------------------- DeepSeek-V3 sizes (sampled tokens)
+
+def _sample(T, n, seed=0):
+    rng = np.random.default_rng(seed)
+    s = set([0, T - 1]) | set(rng.choice(T, min(n, T), replace=False).tolist())
+    return np.array(sorted(s), dtype=np.int32)
+
+
+@pytest.mark.parametrize("T", [128, 1, 37])
+def test_decode(T):
+    wl = WORKLOADS["decode"]
+    W = inputs("decode", "cuda")
+    x = make_x(wl, "cuda", T=T) if T != wl.T else W["x"]
+    toks = _sample(T, 6)
+    ref = oracle_y(wl, W, x, toks)
+    y = run_forward(wl, W, x, torch.float32)
+    assert_close_rms(y.cpu().numpy()[toks], ref, REL)
+    yb = run_forward(wl, W, x, torch.bfloat16)
+    assert_close_bf16(yb[torch.from_numpy(toks).long().to(DEV)], ref, REL)
+
+
+def test_prefill_sampled():
+    wl = WORKLOADS["prefill"]
+    W = inputs("prefill", "cuda")
+    x = W["x"]
+    toks = _sample(wl.T, 6, seed=1)
+    ref = oracle_y(wl, W, x, toks)
+    yb = run_forward(wl, W, x, torch.bfloat16)
+    assert_close_bf16(yb[torch.from_numpy(toks).long().to(DEV)], ref, REL)
+
+
+def test_skewed_sampled():
+    wl = WORKLOADS["skewed"]
+    W = inputs("skewed", "cuda")
+    x = W["x"]
+    toks = _sample(wl.T, 4, seed=2)
+    ref = oracle_y(wl, W, x, toks)
+    y = run_forward(wl, W, x, torch.float32)
+    assert_close_rms(y.cpu().numpy()[toks], ref, REL)
