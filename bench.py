@@ -1,0 +1,459 @@
+#!/usr/bin/env python
+"""Benchmark of the DeepSeek-V3 MoE layer forward pass on B200.
+
+One step = one moe_forward (router, group-limited top-8 selection, permutation,
+256 routed SwiGLU experts + the shared expert, weighted combine) over one
+batch of T tokens whose inputs are already resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|skewed|fp8|tiny]
+    python bench.py --impl reference ...   # the CPU oracle on a bounded sample
+
+With N > 1 (launched by torchrun) every rank runs an independent replica of
+the layer on its own GPU and batch (weak scaling; the layer has no exchange
+step on one node without expert parallelism).  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/sec (T=128 decode, T=4096 prefill); % of HBM/tensor roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS_PER_STEP = 7  # router, select, permute, gather, gate/up GEMM, down GEMM, cast
+
+# DRAM traffic of the dominant kernel per launch, from one ncu capture, keyed by
+# workload; valid only while the kernel sources hash to the recorded value.
+NCU_TRAFFIC = {}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "fine_grained_moe_gemm_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(open(os.path.join(d, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return {k: float(j[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (read-only) while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            try:
+                bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._nv = pynvml
+        except Exception:
+            self._h = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                util = nv.nvmlDeviceGetUtilizationRates(self._h).gpu
+                self.samples.append((mhz, r, util))
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._h is not None:
+            self._t.join()
+
+    def summary(self):
+        if self._h is None or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": len(self.samples)}
+        busy = [s for s in self.samples if s[2] > 0] or self.samples
+        bits = 0
+        for s in busy:
+            bits |= s[1]
+        names = [n for b, n in self.REASONS.items() if bits & b and b != 0x1]
+        return {"sm_mhz": statistics.median(s[0] for s in busy), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(busy)}
+
+
+# --------------------------------------------------------------------------- accounting
+def layer_accounting(wl, T, U, out_bytes):
+    """Algorithmic flops / bytes of one layer step: the weights of the U touched
+    routed experts + the shared expert + the router, x read once, y written once."""
+    wb = 1 if wl.fp8 else 2
+    F = T * wl.flops_per_token
+    B = ((U + 1) * 3 * wl.hidden * wl.d * wb + wl.n_experts * wl.d * 2 + T * wl.d * 2 + T * wl.d * out_bytes)
+    if wl.fp8:
+        B += (U + 1) * 3 * (wl.hidden // 128) * (wl.d // 128) * 4
+    return F, B
+
+
+def kernel_accounting(wl, T, U, stage):
+    """Algorithmic flops / bytes of one launch of a grouped GEMM.
+    gate_up: gate+up weights of the touched experts, the permuted x rows read
+    once, h written once.  down: down weights, h read once, fp32 combine
+    buffer written once."""
+    wb = 1 if wl.fp8 else 2
+    rows = T * wl.top_k + T
+    if stage == "gate_up":
+        F = rows * 2 * 2 * wl.hidden * wl.d
+        B = (U + 1) * 2 * wl.hidden * wl.d * wb + rows * wl.d * 2 + rows * wl.hidden * 2
+    else:
+        F = rows * 2 * wl.hidden * wl.d
+        B = (U + 1) * wl.hidden * wl.d * wb + rows * wl.hidden * 2 + T * wl.d * 4
+    return F, B
+
+
+def roofline(F, B, seconds, peaks, peak_kind):
+    t_tc = F / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = B / (peaks["hbm_gbs"] * 1e9)
+    if t_hbm >= t_tc:
+        ach = B / seconds / 1e9
+        return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(ach / peaks["hbm_gbs"], 4), "peak_source": peak_kind}
+    ach = F / seconds / 1e12
+    return {"bound": "tensor", "achieved": round(ach, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": round(ach / peaks["bf16_tflops"], 4), "peak_source": peak_kind}
+
+
+# --------------------------------------------------------------------------- oracle timing
+def _oracle_runner(wl, W, x, n_tokens):
+    """An oracle run on n_tokens of the batch (the CPU oracle alone; nothing of
+    the CUDA path).  The sampled tokens are chosen, among the first 64, to
+    share experts: that keeps the host copy of the weights small and leaves the
+    per-token cost unchanged (every token evaluates its routing plus k routed
+    experts and the shared expert).  Returns (run, n, threads)."""
+    import numpy as np
+    import torch
+
+    import oracle
+
+    T = x.shape[0]
+    pool = min(T, 64)
+
+    def u16(t):
+        return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+    def u8(t):
+        return t.detach().contiguous().view(torch.uint8).cpu().numpy()
+
+    xp = x[:pool]
+    xp_h = xp.cpu().numpy() if xp.dtype == torch.float32 else u16(xp)
+    wr_h = u16(W["w_router"])
+    bias_h = W["bias"].cpu().numpy()
+    idx_h, _ = oracle.select(oracle.router_logits(xp_h, wr_h), bias_h, wl.n_groups, wl.topk_groups, wl.top_k)
+    chosen, experts = [], set()
+    while len(chosen) < min(n_tokens, pool):
+        best = min((t for t in range(pool) if t not in chosen), key=lambda t: (len(set(idx_h[t]) - experts), t))
+        chosen.append(best)
+        experts |= set(idx_h[best].tolist())
+    toks = np.array(sorted(chosen), dtype=np.int32)
+    xs_h = xp_h[toks]
+
+    conv = u8 if wl.fp8 else u16
+    E = wl.n_experts
+    wg, wu, wd = [None] * E, [None] * E, [None] * E
+    kw = {}
+    if wl.fp8:
+        sg, su, sd = [None] * E, [None] * E, [None] * E
+    for e in sorted(experts):
+        wg[e], wu[e], wd[e] = conv(W["w_gate"][e]), conv(W["w_up"][e]), conv(W["w_down"][e])
+        if wl.fp8:
+            sg[e], su[e], sd[e] = (W["s_gate"][e].cpu().numpy(), W["s_up"][e].cpu().numpy(),
+                                   W["s_down"][e].cpu().numpy())
+    if wl.fp8:
+        kw = dict(s_gate=sg, s_up=su, s_down=sd, ss_gate=W["ss_gate"].cpu().numpy(),
+                  ss_up=W["ss_up"].cpu().numpy(), ss_down=W["ss_down"].cpu().numpy())
+    L = oracle.Layer(wl.d, E, wl.hidden, wl.shared_hidden, wl.top_k, wl.routed_scale, wg, wu, wd,
+                     conv(W["ws_gate"]), conv(W["ws_up"]), conv(W["ws_down"]), x_is_f32=wl.x_f32, **kw)
+    threads = max(1, min(os.cpu_count() or 1, len(toks)))
+
+    def run():
+        # the oracle's whole path on the sampled tokens: router logits (fp64),
+        # selection, permutation, experts and combine
+        l = oracle.router_logits(xs_h, wr_h)
+        i2, w2 = oracle.select(l, bias_h, wl.n_groups, wl.topk_groups, wl.top_k)
+        oracle.permute(i2, wl.n_experts)
+        oracle.expert_tokens(L, xs_h, i2, w2, np.arange(len(toks)), n_threads=threads)
+
+    return run, len(toks), threads
+
+
+def _cfg(wl):
+    import fine_grained_moe_gemm_b200 as moe
+    return moe.MoeConfig(wl.d, wl.n_experts, wl.n_groups, wl.topk_groups, wl.top_k, wl.hidden, 1, wl.shared_hidden,
+                         wl.routed_scale, moe.MOE_F32 if wl.x_f32 else moe.MOE_BF16,
+                         moe.MOE_E4M3 if wl.fp8 else moe.MOE_BF16)
+
+
+def workload_desc(wl):
+    w = (f"{wl.name}: DeepSeek-V3 MoE layer forward, T={wl.T}, d={wl.d}, {wl.n_experts} routed experts in "
+         f"{wl.n_groups} groups (top-{wl.topk_groups} groups, top-{wl.top_k} experts), SwiGLU hidden {wl.hidden}, "
+         f"1 shared expert (hidden {wl.shared_hidden}), routed scale {wl.routed_scale}")
+    if wl.fp8:
+        w += ", e4m3 expert weights with 128x128 fp32 block scales, activations e4m3 per 1x128"
+    if wl.bias == "hot":
+        w += f", selection bias +{wl.hot_bias} on {wl.n_hot} Zipf({wl.zipf_s}) hot experts"
+    elif wl.bias == "zero":
+        w += ", selection bias 0"
+    else:
+        w += ", selection bias U[-0.1, 0.1]"
+    return w
+
+
+# --------------------------------------------------------------------------- arms
+def run_reference(args, wl):
+    """The CPU oracle, as it stands, on the host cores: each step is a bounded
+    sample of the batch (see cpu_baseline.sample)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+
+    from workloads import make_inputs
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    if dev == "cpu" and wl.d > 1024:
+        print(json.dumps({"impl": "reference", "unavailable": "full-size synthetic weights are generated on a GPU"}))
+        return 0
+    W = make_inputs(wl, dev)
+    W = {k: v.to("cuda") for k, v in W.items()} if dev == "cuda" else W
+    n = args.cpu_sample or min(wl.T, 8)
+    run, n, threads = _oracle_runner(wl, W, W["x"], n)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    sample = (f"{n} of the {wl.T} tokens per step (tokens chosen to share experts; every token costs k routed + "
+              f"1 shared expert evaluations plus its routing)")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": workload_desc(wl), "T": wl.T},
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def run_ours(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    import fine_grained_moe_gemm_b200 as moe
+    from workloads import make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    peaks, peak_kind = load_peaks()
+    cfg = _cfg(wl)
+    T = wl.T
+    src_dev = "cpu" if wl.d <= 1024 else dev
+    W = {k: v.to(dev) for k, v in make_inputs(wl, src_dev, seed=rank).items()}
+    weights = {k: v for k, v in W.items() if k not in ("x", "bias")}
+    x, bias = W["x"], W["bias"]
+    ws = torch.empty(moe.workspace_size(cfg, T), dtype=torch.uint8, device=dev)
+    y = torch.empty((T, wl.d), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        moe.moe_forward(cfg, weights, x, bias, y, workspace=ws, stage_events=ev)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    if moe.device_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = t_start.elapsed_time(t_end)
+    stage_ms = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+                for i, name in enumerate(moe.STAGES)}
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    if moe.device_error() != 0:
+        raise RuntimeError("device error word set during the timed steps")
+
+    # end to end through the public API with host buffers: pinned x in, y out
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty((T, wl.d), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    e2e_steps = max(1, args.steps)
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        moe.moe_forward(cfg, weights, x_dev, bias, y, workspace=ws)
+        y_host.copy_(y, non_blocking=True)
+
+    for _ in range(max(args.warmup, 1)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item())
+
+    # routed experts actually touched (for the byte accounting), through the ABI
+    logits = torch.empty((T, wl.n_experts), dtype=torch.float32, device=dev)
+    idx = torch.empty((T, wl.top_k), dtype=torch.int32, device=dev)
+    wsel = torch.empty((T, wl.top_k), dtype=torch.float32, device=dev)
+    moe.moe_route(cfg, x, W["w_router"], logits, bias, idx, wsel)
+    counts = torch.empty(wl.n_experts, dtype=torch.int32, device=dev)
+    offs = torch.empty(wl.n_experts + 1, dtype=torch.int32, device=dev)
+    srcp = torch.empty(T * wl.top_k, dtype=torch.int32, device=dev)
+    invp = torch.empty(T * wl.top_k, dtype=torch.int32, device=dev)
+    moe.moe_permute(cfg, idx, counts, offs, srcp, invp)
+    c = counts.cpu()
+    U = int((c > 0).sum())
+
+    line = None
+    if rank == 0:
+        F, B = layer_accounting(wl, T, U, 2)
+        step_s = ms_max / args.steps / 1e3
+        k_name = max(("gate_up", "down+combine"), key=lambda n: stage_ms[n])
+        kF, kB = kernel_accounting(wl, T, U, "gate_up" if k_name == "gate_up" else "down")
+        kr = roofline(kF, kB, stage_ms[k_name] / 1e3, peaks, peak_kind)
+        tr = NCU_TRAFFIC.get(wl.name)
+        kr["traffic"] = tr[0] if tr and tr[1] == kernel_source_hash() else None
+        kr["kernel"] = "moe_gemm_kernel<GATEUP>" if k_name == "gate_up" else "moe_gemm_kernel<DOWN>"
+        lr = roofline(F, B, step_s, peaks, peak_kind)
+        t_roof = max(F / (peaks["bf16_tflops"] * 1e12), B / (peaks["hbm_gbs"] * 1e9))
+        lr["roofline_ms"] = round(t_roof * 1e3, 4)
+        lr["frac_of_roofline_time"] = round(t_roof / step_s, 4)
+        lr["algorithmic_bytes"] = B
+        lr["algorithmic_flops"] = F
+        kr["algorithmic_bytes"] = kB
+        kr["algorithmic_flops"] = kF
+        value = world * T * args.steps / (ms_max / 1e3)
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if wl.fp8 else "bf16",
+            "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights; no checkpoint)",
+            "config": {"workload": workload_desc(wl), "T": T, "experts_touched": U,
+                       "max_rows_per_expert": int(c.max()), "l2": "inputs larger than L2: the touched expert "
+                       f"weights ({(U + 1) * 3 * wl.hidden * wl.d * (1 if wl.fp8 else 2) / 1e9:.2f} GB) stream "
+                       "from HBM every step", "parallelism": f"replicas x{world} (no data-path collective)"},
+            "roofline": kr,
+            "layer_roofline": lr,
+            "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+            "e2e": {"value": round(world * T * e2e_steps / (e2e_ms / 1e3), 1), "unit": UNIT,
+                    "h2d_bytes_per_step": x.numel() * x.element_size(),
+                    "d2h_bytes_per_step": y.numel() * y.element_size()},
+            "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "clocks": clk.summary(),
+            "kernel_source": kernel_source_hash(),
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            n = args.cpu_sample or min(T, 8)
+            run, n, threads = _oracle_runner(wl, W, x, n)
+            t0 = time.perf_counter()
+            run()
+            dt = time.perf_counter() - t0
+            line["cpu_baseline"] = {"value": round(n / dt, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
+                                    "sample": f"{n} of the {T} tokens (chosen to share experts; every token costs "
+                                              "its routing plus k routed + 1 shared expert evaluations), fp64"}
+        print(json.dumps(line))
+    return 0
+
+
+def main():
+    from workloads import WORKLOADS
+
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    p.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
+    p.add_argument("--cpu-sample", type=int, default=0, help="tokens of the oracle sample (0: min(T, 8))")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    args = p.parse_args()
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -74,6 +74,9 @@ def lib():
             L.moe_forward.restype = I
             L.moe_forward.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, I, P, I, I, P,
                                       ctypes.c_size_t, P]
+            L.moe_forward_ex.restype = I
+            L.moe_forward_ex.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, I, P, I, I, P,
+                                         ctypes.c_size_t, P, P]
             L.moe_device_error.restype = I
             L.moe_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), P]
             L.moe_status_string.restype = ctypes.c_char_p
@@ -158,16 +161,33 @@ def make_weights(w: dict) -> MoeWeights:
     return mw
 
 
-def moe_forward(cfg: MoeConfig, weights, x, bias, y, accumulate: bool = False, workspace=None, stream=None):
+class MoeStageEvents(ctypes.Structure):
+    _fields_ = [("ev", ctypes.c_void_p * 6)]
+
+
+STAGES = ("route", "permute+gather", "gate_up", "down+combine", "cast")
+
+
+def moe_forward(cfg: MoeConfig, weights, x, bias, y, accumulate: bool = False, workspace=None, stream=None,
+                stage_events=None):
     """y (+)= MoE(x).  ``weights`` is a MoeWeights or a dict of tensors; ``workspace`` a uint8 CUDA tensor of at
-    least ``workspace_size(cfg, T)`` bytes."""
+    least ``workspace_size(cfg, T)`` bytes.  ``stage_events``: optional list of six torch.cuda.Event(
+    enable_timing=True) recorded around the stages (see ``STAGES``)."""
     for n, t in (("x", x), ("bias", bias), ("y", y), ("workspace", workspace)):
         _dev(t, n)
     mw = weights if isinstance(weights, MoeWeights) else make_weights(weights)
     T = x.shape[0]
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    _check(lib().moe_forward(ctypes.byref(cfg), ctypes.byref(mw), _p(x), _p(bias), T, _p(y), _dtype_code(y),
-                             1 if accumulate else 0, _p(workspace), ws_bytes, _stream(stream)), "moe_forward")
+    ev = None
+    if stage_events is not None:
+        ev = MoeStageEvents()
+        for i, e in enumerate(stage_events):
+            if e is not None and e.cuda_event == 0:
+                e.record()  # torch creates the underlying event lazily
+            ev.ev[i] = e.cuda_event if e is not None else None
+    _check(lib().moe_forward_ex(ctypes.byref(cfg), ctypes.byref(mw), _p(x), _p(bias), T, _p(y), _dtype_code(y),
+                                1 if accumulate else 0, _p(workspace), ws_bytes, _stream(stream),
+                                ctypes.byref(ev) if ev is not None else None), "moe_forward")
 
 
 def device_error(stream=None) -> int:

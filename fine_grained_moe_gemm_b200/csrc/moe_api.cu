@@ -259,6 +259,12 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, int T, in
 moe_status moe_forward(const moe_config* cfg, const moe_weights* wt, const void* x, const float* bias, int T,
                        void* y, moe_dtype y_dtype, int accumulate, void* workspace, size_t ws_bytes,
                        moe_stream_t stream) {
+    return moe_forward_ex(cfg, wt, x, bias, T, y, y_dtype, accumulate, workspace, ws_bytes, stream, nullptr);
+}
+
+moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const void* x, const float* bias, int T,
+                          void* y, moe_dtype y_dtype, int accumulate, void* workspace, size_t ws_bytes,
+                          moe_stream_t stream, const moe_stage_events* events) {
     moe_status st = check_config(cfg);
     if (st != MOE_OK) return st;
     if (T < 0 || (y_dtype != MOE_F32 && y_dtype != MOE_BF16) || (accumulate != 0 && accumulate != 1))
@@ -286,9 +292,14 @@ moe_status moe_forward(const moe_config* cfg, const moe_weights* wt, const void*
     const int ldh = H > Hs ? H : Hs;
     const int bn = pick_bn(((long long)T * k + E - 1) / E);
 
+    auto mark = [&](int i) {
+        if (events && events->ev[i]) cudaEventRecord((cudaEvent_t)events->ev[i], s);
+    };
     // (1)+(2) router and selection
+    mark(0);
     st = route_impl(cfg, di, x, wt->w_router, W.logits, bias, T, W.idx, W.w, s);
     if (st != MOE_OK) return st;
+    mark(1);
 
     // (3) permutation + tile schedules
     PermuteArgs pa;
@@ -317,6 +328,7 @@ moe_status moe_forward(const moe_config* cfg, const moe_weights* wt, const void*
     if (launch_gather(x, cfg->act_dtype == MOE_F32, d, W.row_tok, W.row_off + NG, rows_max, W.x_perm, di.sm_count,
                       s) != cudaSuccess)
         return MOE_ERR_CUDA;
+    mark(2);
 
     // (4) gate/up grouped GEMM with the SwiGLU epilogue -> h_perm
     GemmArgs g;
@@ -341,6 +353,7 @@ moe_status moe_forward(const moe_config* cfg, const moe_weights* wt, const void*
     g.h = W.h_perm;
     g.ldh = ldh;
     if (launch_gemm(MODE_GATEUP, bn, &g, di.sm_count, s) != cudaSuccess) return MOE_ERR_CUDA;
+    mark(3);
 
     // (5) down GEMM, routing-weight scale and un-permute scatter into fp32
     float* yacc = y_dtype == MOE_F32 ? static_cast<float*>(y) : W.y_acc;
@@ -371,11 +384,13 @@ moe_status moe_forward(const moe_config* cfg, const moe_weights* wt, const void*
     dn.row_tok = W.row_tok;
     dn.ldy = d;
     if (launch_gemm(MODE_DOWN, bn, &dn, di.sm_count, s) != cudaSuccess) return MOE_ERR_CUDA;
+    mark(4);
 
     if (y_dtype == MOE_BF16 &&
         launch_finalize_bf16(W.y_acc, static_cast<__nv_bfloat16*>(y), (size_t)T * d, accumulate != 0, s) !=
             cudaSuccess)
         return MOE_ERR_CUDA;
+    mark(5);
     return MOE_OK;
 }
 

@@ -159,6 +159,22 @@ MOE_API moe_status moe_forward(const moe_config* cfg, const moe_weights* w, cons
                        int T, void* y, moe_dtype y_dtype, int accumulate, void* workspace,
                        size_t ws_bytes, moe_stream_t stream);
 
+/* Stage timing for moe_forward_ex: six CUDA events (cudaEvent_t handles,
+ * created by the caller) that the call records on `stream`:
+ *   ev[0] before the router          ev[3] after the gate/up GEMM (SwiGLU)
+ *   ev[1] after the selection        ev[4] after the down GEMM and combine
+ *   ev[2] after permutation + gather ev[5] after the output cast
+ * so that cudaEventElapsedTime(ev[i], ev[i+1]) is the device time of a stage. */
+typedef struct CUevent_st* moe_event_t;
+typedef struct {
+    moe_event_t ev[6];
+} moe_stage_events;
+
+/* moe_forward, recording the stage events when `events` is not NULL. */
+MOE_API moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* w, const void* x, const float* bias,
+                                  int T, void* y, moe_dtype y_dtype, int accumulate, void* workspace,
+                                  size_t ws_bytes, moe_stream_t stream, const moe_stage_events* events);
+
 /* Reads and clears the calling thread's current device's error word.  This
  * call synchronises `stream` (it waits for the work enqueued before it).
  * *flags receives the MOE_DEVERR_* bits; returns MOE_ERR_DEVICE if any is set. */
