@@ -175,6 +175,39 @@ MOE_API moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* w, c
                                   int T, void* y, moe_dtype y_dtype, int accumulate, void* workspace,
                                   size_t ws_bytes, moe_stream_t stream, const moe_stage_events* events);
 
+/* Size of the device scratch array that moe_forward_noalloc uses in place of
+ * a caller-provided workspace: 32 MiB.  At the DeepSeek-V3 sizes (d = 7168,
+ * 256 experts, top-8, H = Hs = 2048, one shared expert) that holds up to
+ * T = 170 tokens, which covers decode batches. */
+#define MOE_NOALLOC_MAX_BYTES ((size_t)32 << 20)
+
+/* moe_forward without a workspace argument, for callers that cannot allocate
+ * device memory when they call the layer: for example code that must not
+ * touch the device allocator on its path (cudaMalloc and cudaFree may
+ * synchronise the whole device), or a host that embeds the layer while all
+ * device memory belongs to another program's allocator with no handle it can
+ * lend.  This entry point has no counterpart on the pages; it is a
+ * deployment convenience around moe_forward.
+ *
+ *   - The scratch is one static device array of MOE_NOALLOC_MAX_BYTES per GPU
+ *     that loads the library; it stays allocated until the process exits.
+ *     The call allocates nothing (no cudaMalloc, cudaFree or allocating
+ *     library routine).
+ *   - If moe_workspace_size(cfg, T) exceeds MOE_NOALLOC_MAX_BYTES the call
+ *     returns MOE_ERR_WORKSPACE and enqueues nothing; use moe_forward then.
+ *   - The first call on a device looks up the array's device address for that
+ *     device (cudaGetSymbolAddress, once per device, with the device current);
+ *     make that first call before any stream capture.
+ *   - Every call on a device shares the one array.  Calls whose work overlaps
+ *     on the GPU (other streams, other host threads) race on it and give wrong
+ *     results: order them on one stream or serialise them.  Whatever a
+ *     previous call left in the array does not change a later call's result:
+ *     every value that reaches the output is rewritten or cleared first.
+ * Arguments, layouts and results as moe_forward. */
+MOE_API moe_status moe_forward_noalloc(const moe_config* cfg, const moe_weights* w, const void* x,
+                                       const float* bias, int T, void* y, moe_dtype y_dtype, int accumulate,
+                                       moe_stream_t stream);
+
 /* Reads and clears the calling thread's current device's error word.  This
  * call synchronises `stream` (it waits for the work enqueued before it).
  * *flags receives the MOE_DEVERR_* bits; returns MOE_ERR_DEVICE if any is set. */
