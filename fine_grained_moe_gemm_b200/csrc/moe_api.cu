@@ -103,14 +103,19 @@ bool map_bf16(CUtensorMap* m, const void* p, uint64_t rows, uint64_t cols, uint3
 }
 
 // ------------------------------------------------------------------ tiles
-// Token-chunk width of the grouped GEMMs from the expected rows per expert:
-// small chunks for decode (few tokens per expert), wide ones for prefill.
+// Token-chunk width BN of the grouped GEMMs from the mean rows per expert.
+// An item loads only the rows it has (32-row boxes), so a wide BN costs no
+// traffic, only pipeline depth and TMEM double buffering: small BN for decode
+// (a few tokens per expert, deep pipeline), 256 once experts hold ~100 rows,
+// so that an expert's weights are streamed once and never split in chunks.
 int pick_bn(long long rows_per_expert) {
-    if (rows_per_expert <= 24) return 32;
-    if (rows_per_expert <= 48) return 64;
-    if (rows_per_expert <= 160) return 128;
+    if (rows_per_expert <= 16) return 32;
+    if (rows_per_expert <= 40) return 64;
+    if (rows_per_expert <= 96) return 128;
     return 256;
 }
+
+constexpr int kBoxRows = 32;  // token rows per B-operand TMA box
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -183,11 +188,11 @@ moe_status route_impl(const moe_config* c, const DevInfo& di, const void* x, con
             const int bn = T <= 256 ? 32 : 128;
             if (!map_bf16(&a.a0, w_router, c->n_experts, c->d, 128)) return MOE_ERR_CUDA;
             a.a1 = a.s0 = a.s1 = a.a0;
-            if (!map_bf16(&a.b, x, T, c->d, bn)) return MOE_ERR_CUDA;
+            if (!map_bf16(&a.b, x, T, c->d, kBoxRows)) return MOE_ERR_CUDA;
             a.item_off = nullptr;
             a.n_rows_single = T;
             a.K_routed = a.K_shared = c->d;
-            a.mt_routed = (c->n_experts + 127) / 128;
+            a.mt_routed = (c->n_experts + 255) / 256;
             a.logits = logits;
             a.n_logit_cols = c->n_experts;
             const int items = a.mt_routed * ((T + bn - 1) / bn);
@@ -321,9 +326,9 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     pa.item_off_gu = W.item_gu;
     pa.item_off_dn = W.item_dn;
     pa.bn_gu = pa.bn_dn = bn;
-    pa.mt_gu_routed = H / 64;
-    pa.mt_gu_shared = Hs / 64;
-    pa.mt_dn = d / 128;
+    pa.mt_gu_routed = H / 128;
+    pa.mt_gu_shared = Hs / 128;
+    pa.mt_dn = (d + 255) / 256;
     if (launch_permute(pa, s) != cudaSuccess) return MOE_ERR_CUDA;
     if (launch_gather(x, cfg->act_dtype == MOE_F32, d, W.row_tok, W.row_off + NG, rows_max, W.x_perm, di.sm_count,
                       s) != cudaSuccess)
@@ -333,22 +338,24 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     // (4) gate/up grouped GEMM with the SwiGLU epilogue -> h_perm
     GemmArgs g;
     memset(&g, 0, sizeof(g));
-    if (!map_bf16(&g.a0, wt->w_gate, (uint64_t)E * H, d, 64) || !map_bf16(&g.a1, wt->w_up, (uint64_t)E * H, d, 64))
+    if (!map_bf16(&g.a0, wt->w_gate, (uint64_t)E * H, d, 128) ||
+        !map_bf16(&g.a1, wt->w_up, (uint64_t)E * H, d, 128))
         return MOE_ERR_CUDA;
     if (cfg->n_shared) {
-        if (!map_bf16(&g.s0, wt->ws_gate, Hs, d, 64) || !map_bf16(&g.s1, wt->ws_up, Hs, d, 64)) return MOE_ERR_CUDA;
+        if (!map_bf16(&g.s0, wt->ws_gate, Hs, d, 128) || !map_bf16(&g.s1, wt->ws_up, Hs, d, 128))
+            return MOE_ERR_CUDA;
     } else {
         g.s0 = g.a0;
         g.s1 = g.a1;
     }
-    if (!map_bf16(&g.b, W.x_perm, rows_max, d, bn)) return MOE_ERR_CUDA;
+    if (!map_bf16(&g.b, W.x_perm, rows_max, d, kBoxRows)) return MOE_ERR_CUDA;
     g.item_off = W.item_gu;
     g.row_off = W.row_off;
     g.n_groups = NG;
     g.n_routed = E;
     g.K_routed = g.K_shared = d;
-    g.mt_routed = H / 64;
-    g.mt_shared = Hs / 64;
+    g.mt_routed = H / 128;
+    g.mt_shared = Hs / 128;
     g.rows_per_expert = H;
     g.h = W.h_perm;
     g.ldh = ldh;
@@ -370,14 +377,14 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     }
     dn.a1 = dn.a0;
     dn.s1 = dn.s0;
-    if (!map_bf16(&dn.b, W.h_perm, rows_max, ldh, bn)) return MOE_ERR_CUDA;
+    if (!map_bf16(&dn.b, W.h_perm, rows_max, ldh, kBoxRows)) return MOE_ERR_CUDA;
     dn.item_off = W.item_dn;
     dn.row_off = W.row_off;
     dn.n_groups = NG;
     dn.n_routed = E;
     dn.K_routed = H;
     dn.K_shared = Hs;
-    dn.mt_routed = dn.mt_shared = d / 128;
+    dn.mt_routed = dn.mt_shared = (d + 255) / 256;
     dn.rows_per_expert = d;
     dn.y = yacc;
     dn.row_coef = W.row_coef;

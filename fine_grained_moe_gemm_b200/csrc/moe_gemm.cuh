@@ -5,26 +5,31 @@
 // Formulation (weights as the M operand, tokens as N):
 //   D[f, r] = sum_k A[f, k] * B[r, k]
 // with A the expert weight rows (nn.Linear [out, in], K contiguous) and B the
-// permuted token rows (K contiguous).  One work item is one 128-row weight
-// tile of one expert times up to BN token rows of that expert, over the full K.
+// permuted token rows (K contiguous).  One work item is 256 weight rows (two
+// 128-row tiles, two accumulators) of one expert times up to BN token rows of
+// that expert, over the full K.  Two tiles against one token tile halve the
+// L2 -> SM traffic of the token rows, which every weight tile of the expert
+// re-reads.  The token rows of an item are loaded in 32-row boxes, only as
+// many as the item has, so BN can cover a whole expert at prefill sizes.
 // A persistent CTA per SM walks items i = blockIdx.x, blockIdx.x + gridDim.x, ...
-// Item order inside an expert is weight-tile major and token-chunk minor, so
-// the chunks that share a weight tile run at the same time and hit in L2.
+// Item order inside an expert is weight-block major and token-chunk minor, so
+// chunks that share weights run at the same time and hit in L2.
 //
-// Roles (192 threads, one CTA per SM):
+// Roles (320 threads, one CTA per SM):
 //   warp 0      TMA producer (one lane): A and B k-blocks into a STAGES-deep
 //               ring of 128B-swizzled shared-memory tiles.
-//   warp 1      TMEM allocator; one lane issues tcgen05.mma (M = 128, N = the
-//               item's token count rounded up to 16, K = 16 per instruction)
-//               into one of two TMEM accumulators.
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator (each warp its lane
-//               quarter), then one of
-//     GATEUP  A = 64 gate rows over 64 up rows of the same features; writes
-//             h = SiLU(gate) * up as bf16 [rows, ldh];
-//     DOWN    scales column r by row_coef[r] (routed_scale * w, or 1 for the
-//             shared expert) and adds it into y[row_tok[r], :] (fp32 red.add),
-//             which is the un-permute scatter of the combine;
-//     LOGITS  stores fp32 router logits [T, E].
+//   warp 1      TMEM allocator; one lane issues tcgen05.mma (M = 128 twice,
+//               N = the item's row count rounded up to 16, K = 16 per
+//               instruction) into the item's accumulator pair.
+//   warps 2-9   epilogue, two groups of four (a warp reads the TMEM lane
+//               quarter warp % 4; the groups split the columns):
+//     GATEUP  tile 0 = gate rows, tile 1 = up rows of the same 128 features:
+//             h = SiLU(gate) * up, written as bf16 [rows, ldh];
+//     DOWN    tiles 0/1 = 256 output features; column r is scaled by
+//             row_coef[r] (routed_scale * w, or 1 for the shared expert) and
+//             added into y[row_tok[r], :] (fp32 red.add): the combine's
+//             un-permute scatter;
+//     LOGITS  tiles 0/1 = experts 0-255; stores fp32 router logits [T, E].
 // Every mbarrier wait is bounded (2 s); on expiry the kernel records
 // MOE_DEVERR_TIMEOUT, drains and returns.
 #pragma once
@@ -36,22 +41,29 @@ namespace moe {
 
 enum GemmMode { GEMM_GATEUP = 0, GEMM_DOWN = 1, GEMM_LOGITS = 2 };
 
+constexpr int GEMM_THREADS = 320;
+constexpr int GEMM_EPI_THREADS = 256;
+constexpr int B_BOX_ROWS = 32;
 
 template <int MODE, int BN>
 struct GemmCfg {
-    static constexpr int A_BYTES = 128 * 128;  // 128 rows x 64 bf16
+    static constexpr int A_TILE = 128 * 128;        // 128 rows x 64 bf16
+    static constexpr int A_BYTES = 2 * A_TILE;      // two tiles
     static constexpr int B_BYTES = BN * 128;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int EPI_STRIDE = 33;  // padded fp32 row of the GATEUP staging tile
-    static constexpr int EPI_BYTES = MODE == GEMM_GATEUP ? 128 * EPI_STRIDE * 4 : 0;
     static constexpr int SMEM_LIMIT = 227 * 1024;
-    static constexpr int MISC_BYTES = 1024;  // barriers, TMEM slot, flags
-    static constexpr int STAGES_FIT = (SMEM_LIMIT - 1024 - EPI_BYTES - MISC_BYTES) / STAGE_BYTES;
-    static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
-    static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + MISC_BYTES;
+    static constexpr int MISC_BYTES = 1024;         // barriers, TMEM slot, flags
+    static constexpr int STAGES_FIT = (SMEM_LIMIT - 1024 - MISC_BYTES) / STAGE_BYTES;
+    static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+    static constexpr int ACC_COLS = 2 * BN;         // [tile 0: BN cols][tile 1: BN cols]
+    static constexpr int NUM_ACC = 2 * ACC_COLS <= 512 ? 2 : 1;
+    static constexpr int TMEM_NEED = NUM_ACC * ACC_COLS;
+    static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
+                                     : TMEM_NEED <= 256 ? 256 : 512;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + MISC_BYTES;
     static_assert(STAGES >= 2, "pipeline needs two stages");
     static_assert(BN % 32 == 0 && BN <= 256, "BN");
+    static_assert(TMEM_NEED <= 512, "TMEM");
 };
 
 struct Item {
@@ -93,14 +105,18 @@ __device__ __forceinline__ Item decode_item(const GemmArgs& P, int i) {
     return it;
 }
 
+__device__ __forceinline__ float silu_mul(float g, float u) {
+    // SiLU(g) * u with SiLU(z) = z * sigmoid(z) ("SwiGLU MLP" box)
+    return g < -80.0f ? 0.0f : __fdividef(g, 1.0f + __expf(-g)) * u;
+}
+
 template <int MODE, int BN>
-__global__ void __launch_bounds__(192, 1) moe_gemm_kernel(const __grid_constant__ GemmArgs P) {
+__global__ void __launch_bounds__(GEMM_THREADS, 1) moe_gemm_kernel(const __grid_constant__ GemmArgs P) {
     using C = GemmCfg<MODE, BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* ring = smem;
-    float* epi = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::EPI_BYTES);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
     uint64_t* full = bars;
     uint64_t* empty = bars + C::STAGES;
     uint64_t* tfull = bars + 2 * C::STAGES;
@@ -120,7 +136,7 @@ __global__ void __launch_bounds__(192, 1) moe_gemm_kernel(const __grid_constant_
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], 4);
+            mbar_init(&tempty[a], GEMM_EPI_THREADS / 32);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -155,24 +171,33 @@ __global__ void __launch_bounds__(192, 1) moe_gemm_kernel(const __grid_constant_
             for (int i = blockIdx.x; i < total; i += gridDim.x) {
                 const Item it = decode_item<BN>(P, i);
                 const int KB = it.K / 64;
-                int arow;
-                if (MODE == GEMM_GATEUP) arow = (it.shared ? 0 : it.g * P.rows_per_expert) + it.m * 64;
-                else arow = (it.shared ? 0 : it.g * P.rows_per_expert) + it.m * 128;
-                const CUtensorMap* ma = it.shared ? &P.s0 : &P.a0;
-                const CUtensorMap* mu = it.shared ? &P.s1 : &P.a1;
+                const int nbox = (it.nvalid + B_BOX_ROWS - 1) / B_BOX_ROWS;
+                const uint32_t bytes = C::A_BYTES + nbox * B_BOX_ROWS * 128;
+                // A rows of the two tiles
+                const CUtensorMap* m0;
+                const CUtensorMap* m1;
+                int r0, r1;
+                const int base = it.shared ? 0 : it.g * P.rows_per_expert;
+                if (MODE == GEMM_GATEUP) {  // gate and up rows of the same 128 features
+                    m0 = it.shared ? &P.s0 : &P.a0;
+                    m1 = it.shared ? &P.s1 : &P.a1;
+                    r0 = r1 = base + it.m * 128;
+                } else {                    // 256 consecutive rows
+                    m0 = m1 = it.shared ? &P.s0 : &P.a0;
+                    r0 = base + it.m * 256;
+                    r1 = r0 + 128;
+                }
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
                     uint8_t* sa = ring + stage * C::STAGE_BYTES;
                     uint8_t* sb = sa + C::A_BYTES;
-                    mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-                    if (MODE == GEMM_GATEUP) {
-                        tma_load_2d(sa, ma, kb * 64, arow, &full[stage], pol_w);
-                        tma_load_2d(sa + 64 * 128, mu, kb * 64, arow, &full[stage], pol_w);
-                    } else {
-                        tma_load_2d(sa, ma, kb * 64, arow, &full[stage], pol_w);
-                    }
-                    tma_load_2d(sb, &P.b, kb * 64, it.row0, &full[stage], pol_x);
+                    mbar_arrive_expect_tx(&full[stage], bytes);
+                    tma_load_2d(sa, m0, kb * 64, r0, &full[stage], pol_w);
+                    tma_load_2d(sa + C::A_TILE, m1, kb * 64, r1, &full[stage], pol_w);
+                    for (int bx = 0; bx < nbox; ++bx)
+                        tma_load_2d(sb + bx * B_BOX_ROWS * 128, &P.b, kb * 64, it.row0 + bx * B_BOX_ROWS,
+                                    &full[stage], pol_x);
                     if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
@@ -194,25 +219,34 @@ __global__ void __launch_bounds__(192, 1) moe_gemm_kernel(const __grid_constant_
                 const uint32_t idesc = idesc_bf16_f32(128, n_mma);
                 if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag)) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                const uint32_t d0 = tmem_base + (uint32_t)(acc * C::ACC_COLS);
+                const uint32_t d1 = d0 + BN;
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait_bounded(&full[stage], phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(ring + stage * C::STAGE_BYTES);
-                    const uint64_t adesc = smem_desc_sw128(a_addr);
+                    const uint64_t adesc0 = smem_desc_sw128(a_addr);
+                    const uint64_t adesc1 = smem_desc_sw128(a_addr + C::A_TILE);
                     const uint64_t bdesc = smem_desc_sw128(a_addr + C::A_BYTES);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        mma_bf16(d_tmem, adesc + 2ull * k, bdesc + 2ull * k, idesc, (kb | k) != 0 ? 1u : 0u);
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t accum = (kb | k) != 0 ? 1u : 0u;
+                        mma_bf16(d0, adesc0 + 2ull * k, bdesc + 2ull * k, idesc, accum);
+                        mma_bf16(d1, adesc1 + 2ull * k, bdesc + 2ull * k, idesc, accum);
+                    }
                     mma_commit(&empty[stage]);
                     issued = true;
                     if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
                 mma_commit(&tfull[acc]);
-                acc ^= 1;
-                if (acc == 0) acc_phase ^= 1u;
+                if (C::NUM_ACC == 2) {
+                    acc ^= 1;
+                    if (acc == 0) acc_phase ^= 1u;
+                } else {
+                    acc_phase ^= 1u;
+                }
             }
             if (*abort_flag && issued) {
                 // let every MMA already issued finish before TMEM is released
@@ -223,70 +257,54 @@ __global__ void __launch_bounds__(192, 1) moe_gemm_kernel(const __grid_constant_
         }
     } else {
         // ---------------------------------------------------- epilogue
-        const int q = warp & 3;          // TMEM lane quarter this warp may read
-        const int et = threadIdx.x - 64; // 0..127
+        const int q = warp & 3;                  // TMEM lane quarter this warp may read
+        const int grp = (warp - 2) >> 2;         // column group: chunks c0 = 32 * (2 i + grp)
+        const int et = threadIdx.x - 64;         // 0..255
         int acc = 0;
         uint32_t acc_phase = 0;
         int n_done = 0;
         for (int i = blockIdx.x; i < total; i += gridDim.x, ++n_done) {
             const Item it = decode_item<BN>(P, i);
-            // one thread waits, all four warps take the same decision (the
-            // GATEUP epilogue synchronises the four warps by named barrier)
+            // one thread waits, all eight warps take the same decision
             if (et == 0) epi_ok[n_done & 1] = mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag) ? 1 : 0;
-            named_bar_sync(1, 128);
+            named_bar_sync(1, GEMM_EPI_THREADS);
             if (!epi_ok[n_done & 1]) break;
             tc_fence_after();
-            const uint32_t tacc = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
-            for (int c0 = 0; c0 < it.nvalid; c0 += 32) {
-                float v[32];
-                tmem_ld32(tacc + (uint32_t)c0, v);
+            const uint32_t t0 = tmem_base + (uint32_t)(acc * C::ACC_COLS) + ((uint32_t)(q * 32) << 16);
+            const uint32_t t1 = t0 + BN;
+            for (int c0 = 32 * grp; c0 < it.nvalid; c0 += 64) {
+                float v0[32], v1[32];
+                tmem_ld32(t0 + (uint32_t)c0, v0);
+                tmem_ld32(t1 + (uint32_t)c0, v1);
                 if (MODE == GEMM_GATEUP) {
-                    // stage [128 lanes][32 cols]: lanes 0-63 gate, 64-127 up
-                    float* row = epi + (q * 32 + lane) * C::EPI_STRIDE;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) row[j] = v[j];
-                    named_bar_sync(1, 128);
-                    const int jj = et >> 2;          // token column within the chunk
-                    const int f0 = (et & 3) * 16;    // 16 features
-                    const int j = c0 + jj;
-                    if (j < it.nvalid) {
-                        uint32_t packed[8];
-#pragma unroll
-                        for (int ff = 0; ff < 16; ff += 2) {
-                            float g0 = epi[(f0 + ff) * C::EPI_STRIDE + jj];
-                            float g1 = epi[(f0 + ff + 1) * C::EPI_STRIDE + jj];
-                            float u0 = epi[(64 + f0 + ff) * C::EPI_STRIDE + jj];
-                            float u1 = epi[(64 + f0 + ff + 1) * C::EPI_STRIDE + jj];
-                            float h0 = g0 / (1.0f + __expf(-g0)) * u0;
-                            float h1 = g1 / (1.0f + __expf(-g1)) * u1;
-                            __nv_bfloat162 p2 = __floats2bfloat162_rn(h0, h1);
-                            packed[ff >> 1] = *reinterpret_cast<uint32_t*>(&p2);
-                        }
-                        __nv_bfloat16* dst = P.h + (size_t)(it.row0 + j) * P.ldh + it.m * 64 + f0;
-                        uint4* d4 = reinterpret_cast<uint4*>(dst);
-                        d4[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                        d4[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-                    }
-                    named_bar_sync(1, 128);
-                } else if (MODE == GEMM_DOWN) {
                     const int f = it.m * 128 + q * 32 + lane;
+                    __nv_bfloat16* dst = P.h + (size_t)(it.row0 + c0) * P.ldh + f;
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj)
+                        if (c0 + jj < it.nvalid) dst[(size_t)jj * P.ldh] = __float2bfloat16_rn(silu_mul(v0[jj], v1[jj]));
+                } else if (MODE == GEMM_DOWN) {
+                    const int f0 = it.m * 256 + q * 32 + lane;
+                    const int f1 = f0 + 128;
+                    const bool ok0 = f0 < P.ldy, ok1 = f1 < P.ldy;
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
-                        const int j = c0 + jj;
-                        if (j < it.nvalid) {
-                            const int r = it.row0 + j;
+                        if (c0 + jj < it.nvalid) {
+                            const int r = it.row0 + c0 + jj;
                             const float cf = __ldg(&P.row_coef[r]);
-                            const int t = __ldg(&P.row_tok[r]);
-                            atomicAdd(&P.y[(size_t)t * P.ldy + f], v[jj] * cf);
+                            float* yr = P.y + (size_t)__ldg(&P.row_tok[r]) * P.ldy;
+                            if (ok0) atomicAdd(yr + f0, v0[jj] * cf);
+                            if (ok1) atomicAdd(yr + f1, v1[jj] * cf);
                         }
                     }
                 } else {
-                    const int e = it.m * 128 + q * 32 + lane;
-                    if (e < P.n_logit_cols) {
+                    const int e0 = it.m * 256 + q * 32 + lane;
+                    const int e1 = e0 + 128;
 #pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) {
-                            const int j = c0 + jj;
-                            if (j < it.nvalid) P.logits[(size_t)(it.row0 + j) * P.n_logit_cols + e] = v[jj];
+                    for (int jj = 0; jj < 32; ++jj) {
+                        if (c0 + jj < it.nvalid) {
+                            float* lr = P.logits + (size_t)(it.row0 + c0 + jj) * P.n_logit_cols;
+                            if (e0 < P.n_logit_cols) lr[e0] = v0[jj];
+                            if (e1 < P.n_logit_cols) lr[e1] = v1[jj];
                         }
                     }
                 }
@@ -294,8 +312,12 @@ __global__ void __launch_bounds__(192, 1) moe_gemm_kernel(const __grid_constant_
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[acc]);
-            acc ^= 1;
-            if (acc == 0) acc_phase ^= 1u;
+            if (C::NUM_ACC == 2) {
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            } else {
+                acc_phase ^= 1u;
+            }
         }
     }
 

@@ -361,7 +361,7 @@ static cudaError_t launch_gemm_t(const GemmArgs* args, int grid, cudaStream_t s)
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    moe_gemm_kernel<MODE, BN><<<grid, 192, C::SMEM_BYTES, s>>>(*args);
+    moe_gemm_kernel<MODE, BN><<<grid, GEMM_THREADS, C::SMEM_BYTES, s>>>(*args);
     return cudaGetLastError();
 }
 
