@@ -30,6 +30,7 @@ METRIC = "MoE-layer tokens/sec (T=128 decode, T=4096 prefill); % of HBM/tensor r
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNELS_PER_STEP = 7  # router, select, permute, gather, gate/up GEMM, down GEMM, cast
+KERNELS_PER_STEP_FP8 = 8  # + the activation quantisation
 
 # DRAM traffic of the dominant kernel per launch, from one ncu capture, keyed by
 # workload; valid only while the kernel sources hash to the recorded value.
@@ -416,7 +417,7 @@ def run_ours(args, wl):
             "e2e": {"value": round(world * T * e2e_steps / (e2e_ms / 1e3), 1), "unit": UNIT,
                     "h2d_bytes_per_step": x.numel() * x.element_size(),
                     "d2h_bytes_per_step": y.numel() * y.element_size()},
-            "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "gpu_launches": (KERNELS_PER_STEP_FP8 if wl.fp8 else KERNELS_PER_STEP) * args.steps,
             "clocks": clk.summary(),
             "kernel_source": kernel_source_hash(),
         }

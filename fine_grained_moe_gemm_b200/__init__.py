@@ -77,6 +77,8 @@ def lib():
             L.moe_forward_ex.restype = I
             L.moe_forward_ex.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, I, P, I, I, P,
                                          ctypes.c_size_t, P, P]
+            L.moe_quantize_act.restype = I
+            L.moe_quantize_act.argtypes = [P, I, I, P, P, P]
             L.moe_device_error.restype = I
             L.moe_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), P]
             L.moe_status_string.restype = ctypes.c_char_p
@@ -188,6 +190,15 @@ def moe_forward(cfg: MoeConfig, weights, x, bias, y, accumulate: bool = False, w
     _check(lib().moe_forward_ex(ctypes.byref(cfg), ctypes.byref(mw), _p(x), _p(bias), T, _p(y), _dtype_code(y),
                                 1 if accumulate else 0, _p(workspace), ws_bytes, _stream(stream),
                                 ctypes.byref(ev) if ev is not None else None), "moe_forward")
+
+
+def moe_quantize_act(x, q, sx, stream=None):
+    """Per-token, per-128-channel e4m3 quantisation of bf16 x [T, d] into codes q (uint8 [T, d]) and scales sx
+    (fp32 [T, d/128])."""
+    for n, t in (("x", x), ("q", q), ("sx", sx)):
+        _dev(t, n)
+    T, d = x.shape
+    _check(lib().moe_quantize_act(_p(x), T, d, _p(q), _p(sx), _stream(stream)), "moe_quantize_act")
 
 
 def device_error(stream=None) -> int:

@@ -116,8 +116,13 @@ int pick_bn(long long rows_per_expert) {
 }
 
 constexpr int kBoxRows = 32;  // token rows per B-operand TMA box
+constexpr int kFp8MaxBn = 64;  // FP8 GEMMs hold their promoted sums in registers
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool map_u8(CUtensorMap* m, const void* p, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    return map_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p, rows, cols, box_rows, 128);
+}
 
 struct Workspace {
     float* logits;
@@ -132,8 +137,14 @@ struct Workspace {
     int32_t* row_off;
     int32_t* item_gu;
     int32_t* item_dn;
-    __nv_bfloat16* x_perm;
-    __nv_bfloat16* h_perm;
+    __nv_bfloat16* x_perm;   // bf16 weights: permuted activations [rows, d]
+    __nv_bfloat16* h_perm;   // bf16 weights: SwiGLU output [rows, ldh]
+    uint8_t* x_q;            // e4m3 weights: quantised x [T, d] and its scales [T, d/128]
+    float* sx;
+    uint8_t* xq_perm;        // permuted codes [rows, d] and scales [d/128][rows]
+    float* sxT;
+    uint8_t* hq;             // h codes [rows, ldh] and scales [ldh/128][rows]
+    float* shT;
     float* y_acc;
     size_t bytes;
 };
@@ -164,8 +175,17 @@ Workspace layout(const moe_config* c, int T, void* base) {
     w.row_off = (int32_t*)take((NG + 1) * 4);
     w.item_gu = (int32_t*)take((NG + 1) * 4);
     w.item_dn = (int32_t*)take((NG + 1) * 4);
-    w.x_perm = (__nv_bfloat16*)take(rows * (size_t)c->d * 2);
-    w.h_perm = (__nv_bfloat16*)take(rows * ldh * 2);
+    if (c->weight_dtype == MOE_E4M3) {
+        w.x_q = (uint8_t*)take((size_t)T * c->d);
+        w.sx = (float*)take((size_t)T * (c->d / 128) * 4);
+        w.xq_perm = (uint8_t*)take(rows * (size_t)c->d);
+        w.sxT = (float*)take(rows * (size_t)(c->d / 128) * 4);
+        w.hq = (uint8_t*)take(rows * ldh);
+        w.shT = (float*)take(rows * (ldh / 128) * 4);
+    } else {
+        w.x_perm = (__nv_bfloat16*)take(rows * (size_t)c->d * 2);
+        w.h_perm = (__nv_bfloat16*)take(rows * ldh * 2);
+    }
     w.y_acc = (float*)take((size_t)T * c->d * 4);
     w.bytes = off;
     return w;
@@ -239,6 +259,17 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router,
     return route_impl(cfg, di, x, w_router, logits, bias, T, topk_idx, topk_w, (cudaStream_t)stream);
 }
 
+moe_status moe_quantize_act(const void* x, int T, int d, uint8_t* q, float* sx, moe_stream_t stream) {
+    if (T < 0 || d <= 0 || d % 128 != 0) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x || !q || !sx || (reinterpret_cast<uintptr_t>(x) & 7u) || (reinterpret_cast<uintptr_t>(q) & 3u))
+        return MOE_ERR_INVALID_ARG;
+    DevInfo di;
+    moe_status st = check_device(&di);
+    if (st != MOE_OK) return st;
+    return cuda_status(launch_quant_act(static_cast<const __nv_bfloat16*>(x), T, d, q, sx, (cudaStream_t)stream));
+}
+
 moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, int T, int32_t* counts, int32_t* offsets,
                        int32_t* src, int32_t* inv, moe_stream_t stream) {
     moe_status st = check_config(cfg);
@@ -283,7 +314,12 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
         return MOE_ERR_INVALID_ARG;
     if (cfg->n_shared && (!aligned16(wt->ws_gate) || !aligned16(wt->ws_up) || !aligned16(wt->ws_down)))
         return MOE_ERR_INVALID_ARG;
-    if (cfg->weight_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    const bool fp8 = cfg->weight_dtype == MOE_E4M3;
+    if (fp8) {
+        if (cfg->act_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+        if (!wt->s_gate || !wt->s_up || !wt->s_down) return MOE_ERR_INVALID_ARG;
+        if (cfg->n_shared && (!wt->ss_gate || !wt->ss_up || !wt->ss_down)) return MOE_ERR_INVALID_ARG;
+    }
     if (ws_bytes < layout(cfg, T, nullptr).bytes) return MOE_ERR_WORKSPACE;
     DevInfo di;
     if ((st = check_device(&di)) != MOE_OK) return st;
@@ -295,7 +331,8 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     const int NG = E + cfg->n_shared;
     const int rows_max = T * k + cfg->n_shared * T;
     const int ldh = H > Hs ? H : Hs;
-    const int bn = pick_bn(((long long)T * k + E - 1) / E);
+    int bn = pick_bn(((long long)T * k + E - 1) / E);
+    if (fp8 && bn > kFp8MaxBn) bn = kFp8MaxBn;
 
     auto mark = [&](int i) {
         if (events && events->ev[i]) cudaEventRecord((cudaEvent_t)events->ev[i], s);
@@ -330,25 +367,33 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     pa.mt_gu_shared = Hs / 128;
     pa.mt_dn = (d + 255) / 256;
     if (launch_permute(pa, s) != cudaSuccess) return MOE_ERR_CUDA;
-    if (launch_gather(x, cfg->act_dtype == MOE_F32, d, W.row_tok, W.row_off + NG, rows_max, W.x_perm, di.sm_count,
-                      s) != cudaSuccess)
+    if (fp8) {
+        if (launch_quant_act(static_cast<const __nv_bfloat16*>(x), T, d, W.x_q, W.sx, s) != cudaSuccess ||
+            launch_gather_fp8(W.x_q, W.sx, d, W.row_tok, W.row_off + NG, rows_max, W.xq_perm, W.sxT, di.sm_count,
+                              s) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    } else if (launch_gather(x, cfg->act_dtype == MOE_F32, d, W.row_tok, W.row_off + NG, rows_max, W.x_perm,
+                             di.sm_count, s) != cudaSuccess) {
         return MOE_ERR_CUDA;
+    }
     mark(2);
 
     // (4) gate/up grouped GEMM with the SwiGLU epilogue -> h_perm
+    auto wmap = [&](CUtensorMap* m, const void* p, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+        return fp8 ? map_u8(m, p, rows, cols, box_rows) : map_bf16(m, p, rows, cols, box_rows);
+    };
     GemmArgs g;
     memset(&g, 0, sizeof(g));
-    if (!map_bf16(&g.a0, wt->w_gate, (uint64_t)E * H, d, 128) ||
-        !map_bf16(&g.a1, wt->w_up, (uint64_t)E * H, d, 128))
+    if (!wmap(&g.a0, wt->w_gate, (uint64_t)E * H, d, 128) || !wmap(&g.a1, wt->w_up, (uint64_t)E * H, d, 128))
         return MOE_ERR_CUDA;
     if (cfg->n_shared) {
-        if (!map_bf16(&g.s0, wt->ws_gate, Hs, d, 128) || !map_bf16(&g.s1, wt->ws_up, Hs, d, 128))
-            return MOE_ERR_CUDA;
+        if (!wmap(&g.s0, wt->ws_gate, Hs, d, 128) || !wmap(&g.s1, wt->ws_up, Hs, d, 128)) return MOE_ERR_CUDA;
     } else {
         g.s0 = g.a0;
         g.s1 = g.a1;
     }
-    if (!map_bf16(&g.b, W.x_perm, rows_max, d, kBoxRows)) return MOE_ERR_CUDA;
+    if (!(fp8 ? map_u8(&g.b, W.xq_perm, rows_max, d, kBoxRows) : map_bf16(&g.b, W.x_perm, rows_max, d, kBoxRows)))
+        return MOE_ERR_CUDA;
     g.item_off = W.item_gu;
     g.row_off = W.row_off;
     g.n_groups = NG;
@@ -359,7 +404,22 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     g.rows_per_expert = H;
     g.h = W.h_perm;
     g.ldh = ldh;
-    if (launch_gemm(MODE_GATEUP, bn, &g, di.sm_count, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (fp8) {
+        g.sa0 = wt->s_gate;
+        g.sa1 = wt->s_up;
+        g.ss0 = cfg->n_shared ? wt->ss_gate : wt->s_gate;
+        g.ss1 = cfg->n_shared ? wt->ss_up : wt->s_up;
+        g.a_rb_routed = H / 128;
+        g.a_rb_shared = Hs / 128;
+        g.sbT = W.sxT;
+        g.sb_ld = rows_max;
+        g.hq = W.hq;
+        g.hsT = W.shT;
+        g.hs_ld = rows_max;
+    }
+    if ((fp8 ? launch_gemm_fp8(MODE_GATEUP, bn, &g, di.sm_count, s) : launch_gemm(MODE_GATEUP, bn, &g, di.sm_count, s)) !=
+        cudaSuccess)
+        return MOE_ERR_CUDA;
     mark(3);
 
     // (5) down GEMM, routing-weight scale and un-permute scatter into fp32
@@ -369,15 +429,16 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
         return MOE_ERR_CUDA;
     GemmArgs dn;
     memset(&dn, 0, sizeof(dn));
-    if (!map_bf16(&dn.a0, wt->w_down, (uint64_t)E * d, H, 128)) return MOE_ERR_CUDA;
+    if (!wmap(&dn.a0, wt->w_down, (uint64_t)E * d, H, 128)) return MOE_ERR_CUDA;
     if (cfg->n_shared) {
-        if (!map_bf16(&dn.s0, wt->ws_down, d, Hs, 128)) return MOE_ERR_CUDA;
+        if (!wmap(&dn.s0, wt->ws_down, d, Hs, 128)) return MOE_ERR_CUDA;
     } else {
         dn.s0 = dn.a0;
     }
     dn.a1 = dn.a0;
     dn.s1 = dn.s0;
-    if (!map_bf16(&dn.b, W.h_perm, rows_max, ldh, kBoxRows)) return MOE_ERR_CUDA;
+    if (!(fp8 ? map_u8(&dn.b, W.hq, rows_max, ldh, kBoxRows) : map_bf16(&dn.b, W.h_perm, rows_max, ldh, kBoxRows)))
+        return MOE_ERR_CUDA;
     dn.item_off = W.item_dn;
     dn.row_off = W.row_off;
     dn.n_groups = NG;
@@ -390,7 +451,16 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     dn.row_coef = W.row_coef;
     dn.row_tok = W.row_tok;
     dn.ldy = d;
-    if (launch_gemm(MODE_DOWN, bn, &dn, di.sm_count, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (fp8) {
+        dn.sa0 = dn.sa1 = wt->s_down;
+        dn.ss0 = dn.ss1 = cfg->n_shared ? wt->ss_down : wt->s_down;
+        dn.a_rb_routed = dn.a_rb_shared = d / 128;
+        dn.sbT = W.shT;
+        dn.sb_ld = rows_max;
+    }
+    if ((fp8 ? launch_gemm_fp8(MODE_DOWN, bn, &dn, di.sm_count, s) : launch_gemm(MODE_DOWN, bn, &dn, di.sm_count, s)) !=
+        cudaSuccess)
+        return MOE_ERR_CUDA;
     mark(4);
 
     if (y_dtype == MOE_BF16 &&

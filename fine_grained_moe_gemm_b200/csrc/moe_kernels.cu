@@ -15,6 +15,7 @@
 
 #include "moe_device.cuh"
 #include "moe_gemm.cuh"
+#include "moe_gemm_fp8.cuh"
 #include "moe_launch.h"
 
 namespace moe {
@@ -318,6 +319,47 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const void* __restrict
     }
 }
 
+// ============================================================================ FP8 activations
+// "Teardown: DeepSeek-V3", section 10: activations scaled in 1x128 tiles.
+// One warp per (token, 128-channel block), 4 channels per lane:
+//   sx = amax / 448 (1 when the block is all zero), q = e4m3_rn_sat(x / sx),
+// with the divides correctly rounded in fp32, so the codes are reproducible.
+__global__ void __launch_bounds__(256) quant_act_kernel(const __nv_bfloat16* __restrict__ x, int T, int d,
+                                                        uint8_t* __restrict__ q, float* __restrict__ sx) {
+    const int nb = d / 128;
+    const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (gw >= (long long)T * nb) return;  // uniform per warp
+    const int t = (int)(gw / nb), b = (int)(gw % nb);
+    const size_t off = (size_t)t * d + (size_t)b * 128 + lane * 4;
+    const uint2 raw = *reinterpret_cast<const uint2*>(x + off);
+    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    const float2 a = __bfloat1622float2(p2[0]), c = __bfloat1622float2(p2[1]);
+    float amax = fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(c.x), fabsf(c.y)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    const uint32_t lo = cvt_e4m3x2(__fdiv_rn(a.y, scale), __fdiv_rn(a.x, scale));
+    const uint32_t hi = cvt_e4m3x2(__fdiv_rn(c.y, scale), __fdiv_rn(c.x, scale));
+    *reinterpret_cast<uint32_t*>(q + off) = lo | (hi << 16);
+    if (lane == 0) sx[(size_t)t * nb + b] = scale;
+}
+
+__global__ void __launch_bounds__(256) gather_fp8_kernel(const uint8_t* __restrict__ xq, const float* __restrict__ sx,
+                                                         int d, const int32_t* __restrict__ row_tok,
+                                                         const int32_t* __restrict__ n_rows_dev, int rows_ld,
+                                                         uint8_t* __restrict__ xpq, float* __restrict__ sxT) {
+    const int n_rows = *n_rows_dev;
+    const int nvec = d / 16, nb = d / 128;
+    for (int r = blockIdx.x; r < n_rows; r += gridDim.x) {
+        const int t = row_tok[r];
+        const uint4* src = reinterpret_cast<const uint4*>(xq + (size_t)t * d);
+        uint4* dst = reinterpret_cast<uint4*>(xpq + (size_t)r * d);
+        for (int v = threadIdx.x; v < nvec; v += blockDim.x) dst[v] = src[v];
+        for (int b = threadIdx.x; b < nb; b += blockDim.x) sxT[(size_t)b * rows_ld + r] = sx[(size_t)t * nb + b];
+    }
+}
+
 // ============================================================================ finalize
 __global__ void __launch_bounds__(256) finalize_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ y,
                                                        size_t n8, int accumulate) {
@@ -397,6 +439,63 @@ cudaError_t launch_gemm(int mode, int bn, const GemmArgs* args, int grid, cudaSt
     if (mode == MODE_GATEUP) return launch_mode<GEMM_GATEUP>(bn, args, grid, s);
     if (mode == MODE_DOWN) return launch_mode<GEMM_DOWN>(bn, args, grid, s);
     return launch_mode<GEMM_LOGITS>(bn, args, grid, s);
+}
+
+template <int MODE, int BN>
+static cudaError_t launch_gemm_fp8_t(const GemmArgs* args, int grid, cudaStream_t s) {
+    using C = Fp8Cfg<MODE, BN>;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(moe_gemm_fp8_kernel<MODE, BN>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    moe_gemm_fp8_kernel<MODE, BN><<<grid, GEMM_THREADS, C::SMEM_BYTES, s>>>(*args);
+    return cudaGetLastError();
+}
+
+int gemm_fp8_smem_bytes(int mode, int bn) {
+    if (mode == MODE_GATEUP)
+        return bn == 32 ? Fp8Cfg<GEMM_GATEUP, 32>::SMEM_BYTES : bn == 64 ? Fp8Cfg<GEMM_GATEUP, 64>::SMEM_BYTES
+                                                                         : Fp8Cfg<GEMM_GATEUP, 128>::SMEM_BYTES;
+    return bn == 32 ? Fp8Cfg<GEMM_DOWN, 32>::SMEM_BYTES : bn == 64 ? Fp8Cfg<GEMM_DOWN, 64>::SMEM_BYTES
+                                                                   : Fp8Cfg<GEMM_DOWN, 128>::SMEM_BYTES;
+}
+
+cudaError_t launch_gemm_fp8(int mode, int bn, const GemmArgs* args, int grid, cudaStream_t s) {
+    if (mode == MODE_GATEUP) {
+        switch (bn) {
+            case 32: return launch_gemm_fp8_t<GEMM_GATEUP, 32>(args, grid, s);
+            case 64: return launch_gemm_fp8_t<GEMM_GATEUP, 64>(args, grid, s);
+            case 128: return launch_gemm_fp8_t<GEMM_GATEUP, 128>(args, grid, s);
+        }
+    } else if (mode == MODE_DOWN) {
+        switch (bn) {
+            case 32: return launch_gemm_fp8_t<GEMM_DOWN, 32>(args, grid, s);
+            case 64: return launch_gemm_fp8_t<GEMM_DOWN, 64>(args, grid, s);
+            case 128: return launch_gemm_fp8_t<GEMM_DOWN, 128>(args, grid, s);
+        }
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_quant_act(const __nv_bfloat16* x, int T, int d, uint8_t* q, float* sx, cudaStream_t s) {
+    const long long warps = (long long)T * (d / 128);
+    const long long blocks = (warps + 7) / 8;
+    quant_act_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, T, d, q, sx);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_fp8(const uint8_t* xq, const float* sx, int d, const int32_t* row_tok,
+                              const int32_t* n_rows_dev, int max_rows, uint8_t* xpq, float* sxT, int n_sm,
+                              cudaStream_t s) {
+    int grid = max_rows < n_sm * 8 ? max_rows : n_sm * 8;
+    if (grid < 1) grid = 1;
+    gather_fp8_kernel<<<grid, 256, 0, s>>>(xq, sx, d, row_tok, n_rows_dev, max_rows, xpq, sxT);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_router_f32(const float* x, const __nv_bfloat16* wr, int T, int d, int E, float* logits,

@@ -32,6 +32,17 @@ struct GemmArgs {
     int ldy;
     float* logits;             // LOGITS output
     int n_logit_cols;
+    // FP8 (e4m3) operands: per-128x128-block weight scales, per-row block scales of B
+    const float* sa0;          // routed A scales, tile 0: [E][a_rb_routed][K/128]
+    const float* sa1;          // routed A scales, tile 1
+    const float* ss0;          // shared expert A scales, tile 0: [a_rb_shared][K/128]
+    const float* ss1;
+    int a_rb_routed, a_rb_shared;  // 128-row scale blocks per routed / shared weight matrix
+    const float* sbT;          // B scales, K-block major: [K/128][sb_ld]
+    int sb_ld;
+    uint8_t* hq;               // GATEUP FP8 output codes [rows, ldh]
+    float* hsT;                // GATEUP FP8 output scales [ldh/128][hs_ld]
+    int hs_ld;
 };
 
 enum { MODE_GATEUP = 0, MODE_DOWN = 1, MODE_LOGITS = 2 };
@@ -69,6 +80,14 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
 // x_perm[r, :] = x[row_tok[r], :] (fp32 input rounded to bf16) for r < row_off[n_groups]
 cudaError_t launch_gather(const void* x, bool x_f32, int d, const int32_t* row_tok, const int32_t* n_rows_dev,
                           int max_rows, __nv_bfloat16* x_perm, int n_sm, cudaStream_t s);
+// q[t, :], sx[t, b]: per-token, per-128-channel e4m3 quantisation of bf16 x
+cudaError_t launch_quant_act(const __nv_bfloat16* x, int T, int d, uint8_t* q, float* sx, cudaStream_t s);
+// xpq[r, :] = xq[row_tok[r], :]; sxT[b][r] = sx[row_tok[r], b] for r < row_off[n_groups]
+cudaError_t launch_gather_fp8(const uint8_t* xq, const float* sx, int d, const int32_t* row_tok,
+                              const int32_t* n_rows_dev, int max_rows, uint8_t* xpq, float* sxT, int n_sm,
+                              cudaStream_t s);
+int gemm_fp8_smem_bytes(int mode, int bn);
+cudaError_t launch_gemm_fp8(int mode, int bn, const GemmArgs* args, int grid, cudaStream_t s);
 // y[i] = bf16(acc[i] (+ y[i]))
 cudaError_t launch_finalize_bf16(const float* acc, __nv_bfloat16* y, size_t n, bool accumulate, cudaStream_t s);
 cudaError_t read_clear_dev_error(unsigned int* flags, cudaStream_t s);

@@ -146,7 +146,11 @@ MOE_API moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, i
  *   y[t] (+)= routed_scale * sum_j w[t,j] * expert_{idx[t,j]}(x[t]) + shared(x[t])
  * expert(x) = W_down (SiLU(W_gate x) * (W_up x)), SiLU(z) = z * sigmoid(z).
  * x: [T, d] cfg->act_dtype (fp32 input is rounded to bf16 for the experts; with
- * E4M3 weights it is quantised to e4m3 per token and 128-channel block).
+ * E4M3 weights x must be bf16 and is quantised to e4m3 per token and
+ * 128-channel block as moe_quantize_act does, the expert GEMMs run on e4m3
+ * tensor cores with the partial sums of every 128-element K block promoted
+ * to fp32 with both block scales, and h is stored as e4m3 with one scale per
+ * row and 128 features).
  * y: [T, d] in y_dtype (MOE_F32 or MOE_BF16); accumulate = 0 overwrites y,
  * accumulate = 1 adds the layer output to y (the residual stream).
  * The expert GEMMs run on tcgen05 tensor cores with fp32 accumulation; h is
@@ -158,6 +162,16 @@ MOE_API moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, i
 MOE_API moe_status moe_forward(const moe_config* cfg, const moe_weights* w, const void* x, const float* bias,
                        int T, void* y, moe_dtype y_dtype, int accumulate, void* workspace,
                        size_t ws_bytes, moe_stream_t stream);
+
+/* Stage 6, FP8 layers ("Teardown: DeepSeek-V3", section 10: activations in
+ * E4M3 scaled per 1x128 tile).  For every token t and 128-channel block b of
+ * x [T, d] bf16 (d % 128 == 0):
+ *   sx[t, b] = amax_b / 448 (1 when the block is all zero)   fp32 [T, d/128]
+ *   q[t, c]  = e4m3_rn_sat(x[t, c] / sx[t, b])               uint8 [T, d]
+ * The divides are correctly rounded fp32 and the conversion rounds to nearest
+ * even with saturation at +-448 (OCP E4M3), so the codes are reproducible bit
+ * for bit.  moe_forward with E4M3 weights runs the same kernel. */
+MOE_API moe_status moe_quantize_act(const void* x, int T, int d, uint8_t* q, float* sx, moe_stream_t stream);
 
 /* Stage timing for moe_forward_ex: six CUDA events (cudaEvent_t handles,
  * created by the caller) that the call records on `stream`:
