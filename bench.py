@@ -148,16 +148,26 @@ def kernel_accounting(wl, T, U, stage):
     return F, B
 
 
-def roofline(F, B, seconds, peaks, peak_kind):
-    t_tc = F / (peaks["bf16_tflops"] * 1e12)
+FP8_OVER_BF16 = 2.0  # nominal dense e4m3 / bf16 tensor throughput ratio (4.5 / 2.25 PFLOP/s)
+
+
+def tensor_peak(peaks, fp8):
+    """Measured bf16 tensor peak (TFLOP/s); an e4m3 contraction takes it times the nominal ratio."""
+    return peaks["bf16_tflops"] * (FP8_OVER_BF16 if fp8 else 1.0)
+
+
+def roofline(F, B, seconds, peaks, peak_kind, fp8=False):
+    ptc = tensor_peak(peaks, fp8)
+    t_tc = F / (ptc * 1e12)
     t_hbm = B / (peaks["hbm_gbs"] * 1e9)
     if t_hbm >= t_tc:
         ach = B / seconds / 1e9
         return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(ach / peaks["hbm_gbs"], 4), "peak_source": peak_kind}
     ach = F / seconds / 1e12
-    return {"bound": "tensor", "achieved": round(ach, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-            "frac": round(ach / peaks["bf16_tflops"], 4), "peak_source": peak_kind}
+    src = peak_kind + (" bf16 x 2 (nominal e4m3/bf16 ratio)" if fp8 else "")
+    return {"bound": "tensor", "achieved": round(ach, 1), "peak": round(ptc, 1), "unit": "TFLOP/s",
+            "frac": round(ach / ptc, 4), "peak_source": src}
 
 
 # --------------------------------------------------------------------------- oracle timing
@@ -389,12 +399,15 @@ def run_ours(args, wl):
         step_s = ms_max / args.steps / 1e3
         k_name = max(("gate_up", "down+combine"), key=lambda n: stage_ms[n])
         kF, kB = kernel_accounting(wl, T, U, "gate_up" if k_name == "gate_up" else "down")
-        kr = roofline(kF, kB, stage_ms[k_name] / 1e3, peaks, peak_kind)
+        kr = roofline(kF, kB, stage_ms[k_name] / 1e3, peaks, peak_kind, fp8=wl.fp8)
         tr = NCU_TRAFFIC.get(wl.name)
         kr["traffic"] = tr[0] if tr and tr[1] == kernel_source_hash() else None
         kr["kernel"] = "moe_gemm_kernel<GATEUP>" if k_name == "gate_up" else "moe_gemm_kernel<DOWN>"
-        lr = roofline(F, B, step_s, peaks, peak_kind)
-        t_roof = max(F / (peaks["bf16_tflops"] * 1e12), B / (peaks["hbm_gbs"] * 1e9))
+        lr = roofline(F, B, step_s, peaks, peak_kind, fp8=wl.fp8)
+        # the router GEMM stays bf16 in the FP8 layer
+        F_router = 2 * T * wl.n_experts * wl.d
+        t_tc = (F - F_router) / (tensor_peak(peaks, wl.fp8) * 1e12) + F_router / (peaks["bf16_tflops"] * 1e12)
+        t_roof = max(t_tc, B / (peaks["hbm_gbs"] * 1e9))
         lr["roofline_ms"] = round(t_roof * 1e3, 4)
         lr["frac_of_roofline_time"] = round(t_roof / step_s, 4)
         lr["algorithmic_bytes"] = B

@@ -274,8 +274,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) moe_gemm_kernel(const __grid_
             const uint32_t t1 = t0 + BN;
             for (int c0 = 32 * grp; c0 < it.nvalid; c0 += 64) {
                 float v0[32], v1[32];
-                tmem_ld32(t0 + (uint32_t)c0, v0);
-                tmem_ld32(t1 + (uint32_t)c0, v1);
+                tmem_ld32x2(t0 + (uint32_t)c0, t1 + (uint32_t)c0, v0, v1);
                 if (MODE == GEMM_GATEUP) {
                     const int f = it.m * 128 + q * 32 + lane;
                     __nv_bfloat16* dst = P.h + (size_t)(it.row0 + c0) * P.ldh + f;

@@ -17,8 +17,10 @@
 //           and 128-feature block (scale = amax / 448), codes [rows, ldh] and
 //           scales transposed [ldh/128][rows] (the down GEMM's B operand);
 //   DOWN    y[row_tok[r], f] += row_coef[r] * D[f, r] (fp32 red.add).
-// BN <= 128: two partial buffers of 2 x BN TMEM columns; each epilogue thread
-// holds 2 x BN/2 fp32 accumulators.
+// BN <= 128: up to four partial buffers of 2 x BN TMEM columns, so that the
+// MMAs run ahead of the promotion; each epilogue warp waits for a partial by
+// itself and the scales of the next K block are loaded while it waits.  Each
+// epilogue thread holds 2 x BN/2 fp32 accumulators.
 #pragma once
 
 #include "moe_gemm.cuh"
@@ -36,7 +38,8 @@ struct Fp8Cfg {
     static constexpr int STAGES_FIT = (SMEM_LIMIT - 1024 - MISC_BYTES) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
     static constexpr int ACC_COLS = 2 * BN;    // one partial buffer: [tile 0: BN][tile 1: BN]
-    static constexpr int TMEM_NEED = 2 * ACC_COLS;
+    static constexpr int NUM_P = 512 / ACC_COLS >= 4 ? 4 : 512 / ACC_COLS;  // partial buffers in TMEM
+    static constexpr int TMEM_NEED = NUM_P * ACC_COLS;
     static constexpr int TMEM_COLS = TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
     static constexpr int CH = BN >= 64 ? BN / 64 : 1;  // column chunks per epilogue thread
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + MISC_BYTES;
@@ -63,11 +66,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) moe_gemm_fp8_kernel(const __g
     uint64_t* full = bars;
     uint64_t* empty = bars + C::STAGES;
     uint64_t* pfull = bars + 2 * C::STAGES;   // partial buffer written
-    uint64_t* pempty = pfull + 2;             // partial buffer consumed
-    uint64_t* drain = pempty + 2;
+    uint64_t* pempty = pfull + C::NUM_P;      // partial buffer consumed
+    uint64_t* drain = pempty + C::NUM_P;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    volatile int* epi_ok = reinterpret_cast<volatile int*>(tmem_slot + 2);  // [2]
+    volatile int* warp_ok = reinterpret_cast<volatile int*>(tmem_slot + 2);  // [8] epilogue warps
     float* sc_rows = reinterpret_cast<float*>(misc + 512);   // [8 warps][2 tiles][32]
     float* amax_x = reinterpret_cast<float*>(misc + 2560);   // [2 groups][4 quarters][32]
 
@@ -79,7 +82,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) moe_gemm_fp8_kernel(const __g
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < C::NUM_P; ++a) {
             mbar_init(&pfull[a], 1);
             mbar_init(&pempty[a], GEMM_EPI_THREADS / 32);
         }
@@ -178,8 +181,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) moe_gemm_fp8_kernel(const __g
                     mma_commit(&pfull[pb]);
                     issued = true;
                     if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
-                    pb ^= 1;
-                    if (pb == 0) pb_phase ^= 1u;
+                    if (++pb == C::NUM_P) { pb = 0; pb_phase ^= 1u; }
                 }
             }
             if (*abort_flag && issued) {
@@ -192,12 +194,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) moe_gemm_fp8_kernel(const __g
         // ---------------------------------------------------- epilogue: promotion + final
         const int q = warp & 3;
         const int grp = (warp - 2) >> 2;
-        const int et = threadIdx.x - 64;
         const int wi = warp - 2;
         float* my_sc = sc_rows + wi * 64;   // [2 tiles][32 columns]
         int pb = 0;
         uint32_t pb_phase = 0;
-        int n_wait = 0;
         bool alive = true;
         for (int i = blockIdx.x; i < total && alive; i += gridDim.x) {
             const Item it = decode_item<BN>(P, i);
@@ -215,43 +215,48 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) moe_gemm_fp8_kernel(const __g
 #pragma unroll
                 for (int j = 0; j < 32; ++j) acc0[c][j] = acc1[c][j] = 0.0f;
 
+            // scales of K block kb: weight blocks of the two tiles, B row of this lane's column
+            auto load_scales = [&](int kb, float& w0, float& w1, float (&xs)[C::CH]) {
+                w0 = rb0 < a_rb ? __ldg(&sa_t0[(sbase + rb0) * KB + kb]) : 0.0f;
+                w1 = rb1 < a_rb ? __ldg(&sa_t1[(sbase + rb1) * KB + kb]) : 0.0f;
+#pragma unroll
+                for (int c = 0; c < C::CH; ++c) {
+                    const int col = 32 * grp + 64 * c + lane;
+                    xs[c] = col < it.nvalid ? __ldg(&P.sbT[(size_t)kb * P.sb_ld + it.row0 + col]) : 0.0f;
+                }
+            };
+            float nw0, nw1, nxs[C::CH];
+            load_scales(0, nw0, nw1, nxs);
             for (int kb = 0; kb < KB; ++kb) {
-                if (et == 0) epi_ok[n_wait & 1] = mbar_wait_bounded(&pfull[pb], pb_phase, abort_flag) ? 1 : 0;
-                named_bar_sync(1, GEMM_EPI_THREADS);
-                if (!epi_ok[n_wait & 1]) { alive = false; break; }
-                ++n_wait;
+                const float sw0 = nw0, sw1 = nw1;
+                float xs[C::CH];
+#pragma unroll
+                for (int c = 0; c < C::CH; ++c) xs[c] = nxs[c];
+                if (kb + 1 < KB) load_scales(kb + 1, nw0, nw1, nxs);
+                if (!mbar_wait_bounded(&pfull[pb], pb_phase, abort_flag)) { alive = false; break; }
                 tc_fence_after();
-                const float sw0 = rb0 < a_rb ? __ldg(&sa_t0[(sbase + rb0) * KB + kb]) : 0.0f;
-                const float sw1 = rb1 < a_rb ? __ldg(&sa_t1[(sbase + rb1) * KB + kb]) : 0.0f;
                 const uint32_t t0 = tmem_base + (uint32_t)(pb * C::ACC_COLS) + ((uint32_t)(q * 32) << 16);
 #pragma unroll
                 for (int c = 0; c < C::CH; ++c) {
                     const int c0 = 32 * grp + 64 * c;
                     if (c0 < it.nvalid) {
-                        // column scales of this K block (B rows), times each tile's weight scale
-                        const int col = c0 + lane;
-                        const float sx = col < it.nvalid ? __ldg(&P.sbT[(size_t)kb * P.sb_ld + it.row0 + col]) : 0.0f;
-                        my_sc[lane] = sw0 * sx;
-                        my_sc[32 + lane] = sw1 * sx;
+                        my_sc[lane] = sw0 * xs[c];
+                        my_sc[32 + lane] = sw1 * xs[c];
                         __syncwarp();
-                        float p[32];
-                        tmem_ld32(t0 + (uint32_t)c0, p);
+                        float p0[32], p1[32];
+                        tmem_ld32x2(t0 + (uint32_t)c0, t0 + BN + (uint32_t)c0, p0, p1);
 #pragma unroll
                         for (int j = 0; j < 32; j += 4) {
-                            const float4 s4 = *reinterpret_cast<const float4*>(my_sc + j);
-                            acc0[c][j + 0] = fmaf(p[j + 0], s4.x, acc0[c][j + 0]);
-                            acc0[c][j + 1] = fmaf(p[j + 1], s4.y, acc0[c][j + 1]);
-                            acc0[c][j + 2] = fmaf(p[j + 2], s4.z, acc0[c][j + 2]);
-                            acc0[c][j + 3] = fmaf(p[j + 3], s4.w, acc0[c][j + 3]);
-                        }
-                        tmem_ld32(t0 + BN + (uint32_t)c0, p);
-#pragma unroll
-                        for (int j = 0; j < 32; j += 4) {
-                            const float4 s4 = *reinterpret_cast<const float4*>(my_sc + 32 + j);
-                            acc1[c][j + 0] = fmaf(p[j + 0], s4.x, acc1[c][j + 0]);
-                            acc1[c][j + 1] = fmaf(p[j + 1], s4.y, acc1[c][j + 1]);
-                            acc1[c][j + 2] = fmaf(p[j + 2], s4.z, acc1[c][j + 2]);
-                            acc1[c][j + 3] = fmaf(p[j + 3], s4.w, acc1[c][j + 3]);
+                            const float4 s0 = *reinterpret_cast<const float4*>(my_sc + j);
+                            const float4 s1 = *reinterpret_cast<const float4*>(my_sc + 32 + j);
+                            acc0[c][j + 0] = fmaf(p0[j + 0], s0.x, acc0[c][j + 0]);
+                            acc0[c][j + 1] = fmaf(p0[j + 1], s0.y, acc0[c][j + 1]);
+                            acc0[c][j + 2] = fmaf(p0[j + 2], s0.z, acc0[c][j + 2]);
+                            acc0[c][j + 3] = fmaf(p0[j + 3], s0.w, acc0[c][j + 3]);
+                            acc1[c][j + 0] = fmaf(p1[j + 0], s1.x, acc1[c][j + 0]);
+                            acc1[c][j + 1] = fmaf(p1[j + 1], s1.y, acc1[c][j + 1]);
+                            acc1[c][j + 2] = fmaf(p1[j + 2], s1.z, acc1[c][j + 2]);
+                            acc1[c][j + 3] = fmaf(p1[j + 3], s1.w, acc1[c][j + 3]);
                         }
                         __syncwarp();
                     }
@@ -259,8 +264,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) moe_gemm_fp8_kernel(const __g
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&pempty[pb]);
-                pb ^= 1;
-                if (pb == 0) pb_phase ^= 1u;
+                if (++pb == C::NUM_P) { pb = 0; pb_phase ^= 1u; }
+            }
+
+            if (MODE == GEMM_GATEUP) {
+                // the final epilogue synchronises the group's four warps: agree
+                // first that none of them gave up on a wait
+                if (lane == 0) warp_ok[wi] = alive ? 1 : 0;
+                named_bar_sync(2 + grp, 128);
+                alive = warp_ok[4 * grp] && warp_ok[4 * grp + 1] && warp_ok[4 * grp + 2] && warp_ok[4 * grp + 3];
             }
             if (!alive) break;
 
