@@ -76,7 +76,7 @@ def lib():
                                       ctypes.c_size_t, P]
             L.moe_forward_ex.restype = I
             L.moe_forward_ex.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, I, P, I, I, P,
-                                         ctypes.c_size_t, P, P]
+                                         ctypes.c_size_t, P, P, P]
             L.moe_quantize_act.restype = I
             L.moe_quantize_act.argtypes = [P, I, I, P, P, P]
             L.moe_device_error.restype = I
@@ -167,14 +167,20 @@ class MoeStageEvents(ctypes.Structure):
     _fields_ = [("ev", ctypes.c_void_p * 6)]
 
 
+class MoeRoutingOut(ctypes.Structure):
+    _fields_ = [("logits", ctypes.c_void_p), ("topk_idx", ctypes.c_void_p), ("topk_w", ctypes.c_void_p)]
+
+
 STAGES = ("route", "permute+gather", "gate_up", "down+combine", "cast")
 
 
 def moe_forward(cfg: MoeConfig, weights, x, bias, y, accumulate: bool = False, workspace=None, stream=None,
-                stage_events=None):
+                stage_events=None, routing_out=None):
     """y (+)= MoE(x).  ``weights`` is a MoeWeights or a dict of tensors; ``workspace`` a uint8 CUDA tensor of at
     least ``workspace_size(cfg, T)`` bytes.  ``stage_events``: optional list of six torch.cuda.Event(
-    enable_timing=True) recorded around the stages (see ``STAGES``)."""
+    enable_timing=True) recorded around the stages (see ``STAGES``).  ``routing_out``: optional dict with any of
+    ``logits`` [T, E] f32, ``topk_idx`` [T, k] int32, ``topk_w`` [T, k] f32 CUDA tensors that receive the routing
+    the layer used."""
     for n, t in (("x", x), ("bias", bias), ("y", y), ("workspace", workspace)):
         _dev(t, n)
     mw = weights if isinstance(weights, MoeWeights) else make_weights(weights)
@@ -187,9 +193,18 @@ def moe_forward(cfg: MoeConfig, weights, x, bias, y, accumulate: bool = False, w
             if e is not None and e.cuda_event == 0:
                 e.record()  # torch creates the underlying event lazily
             ev.ev[i] = e.cuda_event if e is not None else None
+    ro = None
+    if routing_out is not None:
+        ro = MoeRoutingOut()
+        for name in ("logits", "topk_idx", "topk_w"):
+            t = routing_out.get(name)
+            if t is not None:
+                _dev(t, name)
+                setattr(ro, name, t.data_ptr())
     _check(lib().moe_forward_ex(ctypes.byref(cfg), ctypes.byref(mw), _p(x), _p(bias), T, _p(y), _dtype_code(y),
                                 1 if accumulate else 0, _p(workspace), ws_bytes, _stream(stream),
-                                ctypes.byref(ev) if ev is not None else None), "moe_forward")
+                                ctypes.byref(ev) if ev is not None else None,
+                                ctypes.byref(ro) if ro is not None else None), "moe_forward")
 
 
 def moe_quantize_act(x, q, sx, stream=None):

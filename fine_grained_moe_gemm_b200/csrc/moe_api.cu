@@ -120,12 +120,33 @@ constexpr int kFp8MaxBn = 64;  // FP8 GEMMs hold their promoted sums in register
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Router GEMM tiling: token chunk and K splits.  At decode sizes the whole
+// router weight would be streamed by a handful of CTAs; splitting K spreads it
+// over about one item per SM.  The partial logits are summed in a fixed order
+// by the selection kernel, so the logits do not depend on scheduling.
+int router_bn(int T) { return T <= 256 ? 32 : 128; }
+int router_splits(int T, int n_sm) {
+    const int items = (T + router_bn(T) - 1) / router_bn(T);
+    int s = n_sm / items;
+    return s < 1 ? 1 : (s > 16 ? 16 : s);
+}
+// Rows of partial logits to reserve: an upper bound of splits x T that does
+// not decrease with T (a workspace sized for T_max serves every T <= T_max):
+// splits <= 16, and splits x chunks <= 148 when splits > 1.
+size_t router_part_rows(int T) {
+    const size_t t = (size_t)T;
+    if (T <= 256) return t * 16 < 148 * 32 ? t * 16 : 148 * 32;
+    const size_t b = t * 16 < 148 * 128 ? t * 16 : 148 * 128;
+    return b > t ? b : t;
+}
+
 bool map_u8(CUtensorMap* m, const void* p, uint64_t rows, uint64_t cols, uint32_t box_rows) {
     return map_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p, rows, cols, box_rows, 128);
 }
 
 struct Workspace {
     float* logits;
+    float* part;             // split-K partial router logits
     int32_t* idx;
     float* w;
     int32_t* counts;
@@ -164,6 +185,7 @@ Workspace layout(const moe_config* c, int T, void* base) {
         return p;
     };
     w.logits = (float*)take((size_t)T * E * 4);
+    w.part = (float*)take(router_part_rows(T) * E * 4);
     w.idx = (int32_t*)take((size_t)T * k * 4);
     w.w = (float*)take((size_t)T * k * 4);
     w.counts = (int32_t*)take(E * 4);
@@ -195,7 +217,8 @@ moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_E
 
 // Router logits on tensor cores (bf16 x) or CUDA cores (fp32 x), then selection.
 moe_status route_impl(const moe_config* c, const DevInfo& di, const void* x, const void* w_router, float* logits,
-                      const float* bias, int T, int32_t* idx, float* w, cudaStream_t s) {
+                      const float* bias, int T, int32_t* idx, float* w, cudaStream_t s, float* part = nullptr) {
+    int n_parts = 1;
     if (x) {
         if (c->act_dtype == MOE_F32) {
             cudaError_t e = launch_router_f32(static_cast<const float*>(x),
@@ -205,7 +228,9 @@ moe_status route_impl(const moe_config* c, const DevInfo& di, const void* x, con
         } else {
             GemmArgs a;
             memset(&a, 0, sizeof(a));
-            const int bn = T <= 256 ? 32 : 128;
+            const int bn = router_bn(T);
+            if (part && c->n_experts <= 256) n_parts = router_splits(T, di.sm_count);
+            if (n_parts > c->d / 64) n_parts = c->d / 64;  // every split owns at least one K block
             if (!map_bf16(&a.a0, w_router, c->n_experts, c->d, 128)) return MOE_ERR_CUDA;
             a.a1 = a.s0 = a.s1 = a.a0;
             if (!map_bf16(&a.b, x, T, c->d, kBoxRows)) return MOE_ERR_CUDA;
@@ -215,12 +240,15 @@ moe_status route_impl(const moe_config* c, const DevInfo& di, const void* x, con
             a.mt_routed = (c->n_experts + 255) / 256;
             a.logits = logits;
             a.n_logit_cols = c->n_experts;
-            const int items = a.mt_routed * ((T + bn - 1) / bn);
+            a.k_splits = n_parts;
+            a.part = part;
+            const int items = a.mt_routed * ((T + bn - 1) / bn) * n_parts;
             const int grid = items < di.sm_count ? items : di.sm_count;
             if (launch_gemm(MODE_LOGITS, bn, &a, grid, s) != cudaSuccess) return MOE_ERR_CUDA;
         }
     }
-    return cuda_status(launch_select(logits, bias, T, c->n_experts, c->n_groups, c->topk_groups, c->top_k, idx, w, s));
+    return cuda_status(launch_select(logits, bias, T, c->n_experts, c->n_groups, c->topk_groups, c->top_k, idx, w, s,
+                                     part, n_parts));
 }
 
 }  // namespace
@@ -295,12 +323,13 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, int T, in
 moe_status moe_forward(const moe_config* cfg, const moe_weights* wt, const void* x, const float* bias, int T,
                        void* y, moe_dtype y_dtype, int accumulate, void* workspace, size_t ws_bytes,
                        moe_stream_t stream) {
-    return moe_forward_ex(cfg, wt, x, bias, T, y, y_dtype, accumulate, workspace, ws_bytes, stream, nullptr);
+    return moe_forward_ex(cfg, wt, x, bias, T, y, y_dtype, accumulate, workspace, ws_bytes, stream, nullptr,
+                          nullptr);
 }
 
 moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const void* x, const float* bias, int T,
                           void* y, moe_dtype y_dtype, int accumulate, void* workspace, size_t ws_bytes,
-                          moe_stream_t stream, const moe_stage_events* events) {
+                          moe_stream_t stream, const moe_stage_events* events, const moe_routing_out* routing) {
     moe_status st = check_config(cfg);
     if (st != MOE_OK) return st;
     if (T < 0 || (y_dtype != MOE_F32 && y_dtype != MOE_BF16) || (accumulate != 0 && accumulate != 1))
@@ -325,7 +354,17 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     if ((st = check_device(&di)) != MOE_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
 
-    const Workspace W = layout(cfg, T, workspace);
+    Workspace W = layout(cfg, T, workspace);
+    if (routing) {
+        if ((routing->logits && (reinterpret_cast<uintptr_t>(routing->logits) & 3u)) ||
+            (routing->topk_idx && (reinterpret_cast<uintptr_t>(routing->topk_idx) & 3u)) ||
+            (routing->topk_w && (reinterpret_cast<uintptr_t>(routing->topk_w) & 3u)))
+            return MOE_ERR_INVALID_ARG;
+        // the layer routes through the caller's buffers instead of the workspace
+        if (routing->logits) W.logits = routing->logits;
+        if (routing->topk_idx) W.idx = routing->topk_idx;
+        if (routing->topk_w) W.w = routing->topk_w;
+    }
     const int E = cfg->n_experts, k = cfg->top_k, d = cfg->d, H = cfg->hidden;
     const int Hs = cfg->n_shared ? cfg->shared_hidden : H;
     const int NG = E + cfg->n_shared;
@@ -339,7 +378,7 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     };
     // (1)+(2) router and selection
     mark(0);
-    st = route_impl(cfg, di, x, wt->w_router, W.logits, bias, T, W.idx, W.w, s);
+    st = route_impl(cfg, di, x, wt->w_router, W.logits, bias, T, W.idx, W.w, s, W.part);
     if (st != MOE_OK) return st;
     mark(1);
 

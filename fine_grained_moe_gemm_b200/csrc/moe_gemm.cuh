@@ -29,7 +29,9 @@
 //             row_coef[r] (routed_scale * w, or 1 for the shared expert) and
 //             added into y[row_tok[r], :] (fp32 red.add): the combine's
 //             un-permute scatter;
-//     LOGITS  tiles 0/1 = experts 0-255; stores fp32 router logits [T, E].
+//     LOGITS  tiles 0/1 = experts 0-255; stores fp32 router logits [T, E], or,
+//             with K split over several items, one partial per split (summed
+//             in a fixed order by the selection kernel).
 // Every mbarrier wait is bounded (2 s); on expiry the kernel records
 // MOE_DEVERR_TIMEOUT, drains and returns.
 #pragma once
@@ -68,14 +70,22 @@ struct GemmCfg {
 
 struct Item {
     int g, m, row0, nvalid, K;
+    int split, n_splits;  // K range of the item: blocks [split, split+1) * KB / n_splits
     bool shared;
 };
+
+// First and one-past-last K block of an item with KB blocks in all.
+__device__ __forceinline__ int item_kb0(const Item& it, int KB) { return it.split * KB / it.n_splits; }
+__device__ __forceinline__ int item_kb1(const Item& it, int KB) { return (it.split + 1) * KB / it.n_splits; }
 
 template <int BN>
 __device__ __forceinline__ Item decode_item(const GemmArgs& P, int i) {
     Item it;
     if (P.item_off == nullptr) {
         int nch = (P.n_rows_single + BN - 1) / BN;
+        it.n_splits = P.k_splits > 1 ? P.k_splits : 1;
+        it.split = i % it.n_splits;
+        i /= it.n_splits;
         it.g = 0;
         it.m = i / nch;
         int c = i - it.m * nch;
@@ -92,6 +102,8 @@ __device__ __forceinline__ Item decode_item(const GemmArgs& P, int i) {
         else hi = mid - 1;
     }
     it.g = lo;
+    it.split = 0;
+    it.n_splits = 1;
     int local = i - __ldg(&P.item_off[lo]);
     int r0 = __ldg(&P.row_off[lo]);
     int ng = __ldg(&P.row_off[lo + 1]) - r0;
@@ -158,7 +170,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) moe_gemm_kernel(const __grid_
     const uint32_t tmem_base = *tmem_slot;
 
     int total;
-    if (P.item_off == nullptr) total = P.mt_routed * ((P.n_rows_single + BN - 1) / BN);
+    if (P.item_off == nullptr)
+        total = P.mt_routed * ((P.n_rows_single + BN - 1) / BN) * (P.k_splits > 1 ? P.k_splits : 1);
     else total = __ldg(&P.item_off[P.n_groups]);
 
     if (warp == 0) {
@@ -170,7 +183,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) moe_gemm_kernel(const __grid_
             uint32_t phase = 0;
             for (int i = blockIdx.x; i < total; i += gridDim.x) {
                 const Item it = decode_item<BN>(P, i);
-                const int KB = it.K / 64;
+                const int kb0 = item_kb0(it, it.K / 64), kb1 = item_kb1(it, it.K / 64);
                 const int nbox = (it.nvalid + B_BOX_ROWS - 1) / B_BOX_ROWS;
                 const uint32_t bytes = C::A_BYTES + nbox * B_BOX_ROWS * 128;
                 // A rows of the two tiles
@@ -188,7 +201,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) moe_gemm_kernel(const __grid_
                     r1 = r0 + 128;
                 }
                 bool ok = true;
-                for (int kb = 0; kb < KB; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
                     uint8_t* sa = ring + stage * C::STAGE_BYTES;
                     uint8_t* sb = sa + C::A_BYTES;
@@ -213,7 +226,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) moe_gemm_kernel(const __grid_
             bool issued = false;
             for (int i = blockIdx.x; i < total; i += gridDim.x) {
                 const Item it = decode_item<BN>(P, i);
-                const int KB = it.K / 64;
+                const int kb0 = item_kb0(it, it.K / 64), kb1 = item_kb1(it, it.K / 64);
                 uint32_t n_mma = (uint32_t)((it.nvalid + 15) & ~15);
                 n_mma = n_mma < 16u ? 16u : n_mma;
                 const uint32_t idesc = idesc_bf16_f32(128, n_mma);
@@ -222,7 +235,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) moe_gemm_kernel(const __grid_
                 const uint32_t d0 = tmem_base + (uint32_t)(acc * C::ACC_COLS);
                 const uint32_t d1 = d0 + BN;
                 bool ok = true;
-                for (int kb = 0; kb < KB; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait_bounded(&full[stage], phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(ring + stage * C::STAGE_BYTES);
@@ -231,7 +244,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) moe_gemm_kernel(const __grid_
                     const uint64_t bdesc = smem_desc_sw128(a_addr + C::A_BYTES);
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const uint32_t accum = (kb | k) != 0 ? 1u : 0u;
+                        const uint32_t accum = (kb > kb0 || k != 0) ? 1u : 0u;
                         mma_bf16(d0, adesc0 + 2ull * k, bdesc + 2ull * k, idesc, accum);
                         mma_bf16(d1, adesc1 + 2ull * k, bdesc + 2ull * k, idesc, accum);
                     }
@@ -301,7 +314,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) moe_gemm_kernel(const __grid_
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
                         if (c0 + jj < it.nvalid) {
-                            float* lr = P.logits + (size_t)(it.row0 + c0 + jj) * P.n_logit_cols;
+                            float* out = it.n_splits > 1
+                                             ? P.part + (size_t)it.split * P.n_rows_single * P.n_logit_cols
+                                             : P.logits;
+                            float* lr = out + (size_t)(it.row0 + c0 + jj) * P.n_logit_cols;
                             if (e0 < P.n_logit_cols) lr[e0] = v0[jj];
                             if (e1 < P.n_logit_cols) lr[e1] = v1[jj];
                         }

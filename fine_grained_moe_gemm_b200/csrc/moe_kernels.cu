@@ -66,11 +66,12 @@ __device__ __forceinline__ void warp_best(float& v, int& id) {
 
 constexpr int SELECT_WARPS = 8;
 
-__global__ void __launch_bounds__(SELECT_WARPS * 32) select_kernel(const float* __restrict__ logits,
+__global__ void __launch_bounds__(SELECT_WARPS * 32) select_kernel(const float* logits,
                                                                    const float* __restrict__ bias, int T, int E,
                                                                    int G, int topk_groups, int k,
                                                                    int32_t* __restrict__ idx_out,
-                                                                   float* __restrict__ w_out) {
+                                                                   float* __restrict__ w_out,
+                                                                   const float* __restrict__ parts, int n_parts) {
     extern __shared__ float ssm[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.x * SELECT_WARPS + warp;
@@ -79,7 +80,16 @@ __global__ void __launch_bounds__(SELECT_WARPS * 32) select_kernel(const float* 
     float* b = s + E;
     const float* l = logits + (size_t)t * E;
     for (int e = lane; e < E; e += 32) {
-        float sv = sigmoid_spec(l[e]);
+        float lv;
+        if (parts) {
+            // split-K router: the partial logits summed in split order, stored as the logits
+            lv = parts[(size_t)t * E + e];
+            for (int p = 1; p < n_parts; ++p) lv = __fadd_rn(lv, parts[((size_t)p * T + t) * E + e]);
+            const_cast<float*>(l)[e] = lv;
+        } else {
+            lv = l[e];
+        }
+        float sv = sigmoid_spec(lv);
         float bv = __fadd_rn(sv, bias[e]);
         if (bv == 0.0f) bv = 0.0f;
         s[e] = sv;
@@ -505,7 +515,7 @@ cudaError_t launch_router_f32(const float* x, const __nv_bfloat16* wr, int T, in
 }
 
 cudaError_t launch_select(const float* logits, const float* bias, int T, int E, int G, int tg, int k, int32_t* idx,
-                          float* w, cudaStream_t s) {
+                          float* w, cudaStream_t s, const float* parts, int n_parts) {
     const int blocks = (T + SELECT_WARPS - 1) / SELECT_WARPS;
     const size_t smem = (size_t)SELECT_WARPS * 2 * E * sizeof(float);
     static bool attr_set[64] = {};
@@ -517,7 +527,8 @@ cudaError_t launch_select(const float* logits, const float* bias, int T, int E, 
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    select_kernel<<<blocks, SELECT_WARPS * 32, smem, s>>>(logits, bias, T, E, G, tg, k, idx, w);
+    select_kernel<<<blocks, SELECT_WARPS * 32, smem, s>>>(logits, bias, T, E, G, tg, k, idx, w,
+                                                         n_parts > 1 ? parts : nullptr, n_parts);
     return cudaGetLastError();
 }
 

@@ -32,6 +32,8 @@ struct GemmArgs {
     int ldy;
     float* logits;             // LOGITS output
     int n_logit_cols;
+    int k_splits;              // LOGITS: K split over this many items (>= 1)
+    float* part;               // LOGITS with k_splits > 1: partial logits [k_splits][T][E]
     // FP8 (e4m3) operands: per-128x128-block weight scales, per-row block scales of B
     const float* sa0;          // routed A scales, tile 0: [E][a_rb_routed][K/128]
     const float* sa1;          // routed A scales, tile 1
@@ -74,8 +76,9 @@ int gemm_smem_bytes(int mode, int bn);
 cudaError_t launch_gemm(int mode, int bn, const GemmArgs* args, int grid, cudaStream_t s);
 cudaError_t launch_router_f32(const float* x, const __nv_bfloat16* wr, int T, int d, int E, float* logits,
                               cudaStream_t s);
+// parts != nullptr: logits[t, e] = sum over s < n_parts of parts[s][t][e] (fixed order), written first
 cudaError_t launch_select(const float* logits, const float* bias, int T, int E, int G, int tg, int k,
-                          int32_t* idx, float* w, cudaStream_t s);
+                          int32_t* idx, float* w, cudaStream_t s, const float* parts = nullptr, int n_parts = 1);
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
 // x_perm[r, :] = x[row_tok[r], :] (fp32 input rounded to bf16) for r < row_off[n_groups]
 cudaError_t launch_gather(const void* x, bool x_f32, int d, const int32_t* row_tok, const int32_t* n_rows_dev,

@@ -184,15 +184,28 @@ typedef struct {
     moe_event_t ev[6];
 } moe_stage_events;
 
-/* moe_forward, recording the stage events when `events` is not NULL. */
+/* Optional outputs of moe_forward_ex: the routing the layer used.  Each
+ * non-NULL pointer is a caller device buffer that receives the router logits
+ * [T, E] fp32, topk_idx [T, k] int32 or topk_w [T, k] fp32 (unscaled) exactly
+ * as the layer computed and consumed them.  (moe_route runs the router
+ * without splitting K, so its logits may differ from these in the last bits.) */
+typedef struct {
+    float* logits;
+    int32_t* topk_idx;
+    float* topk_w;
+} moe_routing_out;
+
+/* moe_forward, recording the stage events when `events` is not NULL and
+ * writing its routing into `routing` when that is not NULL. */
 MOE_API moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* w, const void* x, const float* bias,
                                   int T, void* y, moe_dtype y_dtype, int accumulate, void* workspace,
-                                  size_t ws_bytes, moe_stream_t stream, const moe_stage_events* events);
+                                  size_t ws_bytes, moe_stream_t stream, const moe_stage_events* events,
+                                  const moe_routing_out* routing);
 
 /* Size of the device scratch array that moe_forward_noalloc uses in place of
  * a caller-provided workspace: 32 MiB.  At the DeepSeek-V3 sizes (d = 7168,
  * 256 experts, top-8, H = Hs = 2048, one shared expert) that holds up to
- * T = 170 tokens, which covers decode batches. */
+ * T = 158 tokens, which covers decode batches. */
 #define MOE_NOALLOC_MAX_BYTES ((size_t)32 << 20)
 
 /* moe_forward without a workspace argument, for callers that cannot allocate

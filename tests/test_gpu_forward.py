@@ -12,7 +12,7 @@ import torch
 
 import oracle
 import fine_grained_moe_gemm_b200 as moe
-from moe_testlib import assert_close_bf16, assert_close_rms, cfg_of, oracle_layer, weights_for_forward, x_host
+from moe_testlib import assert_close_bf16, assert_close_rms, cfg_of, oracle_layer, u16, weights_for_forward, x_host
 from workloads import WORKLOADS, make_inputs, make_residual, make_x
 
 pytestmark = pytest.mark.gpu
@@ -35,34 +35,40 @@ def inputs(name, device_gen):
     return _cache[key]
 
 
-def run_forward(wl, W, x, y_dtype=torch.float32, accumulate=False, y0=None):
+def run_forward(wl, W, x, y_dtype=torch.float32, accumulate=False, y0=None, routing=None):
     cfg = cfg_of(wl)
     T = x.shape[0]
     ws = torch.empty(moe.workspace_size(cfg, T), dtype=torch.uint8, device=DEV)
     y = y0.clone() if y0 is not None else torch.empty((T, wl.d), dtype=y_dtype, device=DEV)
-    moe.moe_forward(cfg, weights_for_forward(W), x, W["bias"], y, accumulate=accumulate, workspace=ws)
+    moe.moe_forward(cfg, weights_for_forward(W), x, W["bias"], y, accumulate=accumulate, workspace=ws,
+                    routing_out=routing)
     torch.cuda.synchronize()
     assert moe.device_error() == 0
     return y
 
 
-def gpu_routing(wl, W, x):
-    cfg = cfg_of(wl)
+def forward_routing(wl, W, x):
+    """The routing moe_forward used (its own logits), checked bit for bit against
+    the oracle's selection on those logits, and its logits against the oracle's
+    fp64 router within tolerance."""
     T = x.shape[0]
-    logits = torch.empty((T, wl.n_experts), dtype=torch.float32, device=DEV)
-    idx = torch.empty((T, wl.top_k), dtype=torch.int32, device=DEV)
-    w = torch.empty((T, wl.top_k), dtype=torch.float32, device=DEV)
-    moe.moe_route(cfg, x, W["w_router"], logits, W["bias"], idx, w)
-    torch.cuda.synchronize()
-    l = logits.cpu().numpy()
+    r = {"logits": torch.empty((T, wl.n_experts), dtype=torch.float32, device=DEV),
+         "topk_idx": torch.empty((T, wl.top_k), dtype=torch.int32, device=DEV),
+         "topk_w": torch.empty((T, wl.top_k), dtype=torch.float32, device=DEV)}
+    run_forward(wl, W, x, routing=r)
+    l = r["logits"].cpu().numpy()
     ridx, rw = oracle.select(l, W["bias"].cpu().numpy(), wl.n_groups, wl.topk_groups, wl.top_k)
-    assert np.array_equal(idx.cpu().numpy(), ridx)
-    assert np.array_equal(w.cpu().numpy().view(np.uint32), rw.view(np.uint32))
+    assert np.array_equal(r["topk_idx"].cpu().numpy(), ridx)
+    assert np.array_equal(r["topk_w"].cpu().numpy().view(np.uint32), rw.view(np.uint32))
+    rows = np.unique(np.linspace(0, T - 1, min(T, 16)).astype(np.int64))
+    l_ref = oracle.router_logits(x_host(x[torch.from_numpy(rows).to(DEV)]), u16(W["w_router"]))
+    rms = float(np.sqrt(np.mean(l_ref.astype(np.float64) ** 2)))
+    assert float(np.max(np.abs(l[rows] - l_ref))) <= 1e-5 * np.sqrt(wl.d) * rms
     return ridx, rw
 
 
 def oracle_y(wl, W, x, tokens):
-    idx, w = gpu_routing(wl, W, x)
+    idx, w = forward_routing(wl, W, x)
     need = np.unique(idx[tokens])
     L = oracle_layer(wl, W, need)
     return oracle.expert_tokens(L, x_host(x), idx, w, tokens)
@@ -134,3 +140,22 @@ def test_skewed_sampled():
     ref = oracle_y(wl, W, x, toks)
     y = run_forward(wl, W, x, torch.float32)
     assert_close_rms(y.cpu().numpy()[toks], ref, REL)
+
+
+def test_forward_routing_repeatable_bitwise():
+    """The split-K router sums its partials in a fixed order: the forward's logits,
+    routing and permutation-dependent output are bit-identical run to run."""
+    wl = WORKLOADS["decode"]
+    W = inputs("decode", "cuda")
+    x = W["x"]
+    T = x.shape[0]
+    outs = []
+    for _ in range(3):
+        r = {"logits": torch.empty((T, wl.n_experts), dtype=torch.float32, device=DEV),
+             "topk_idx": torch.empty((T, wl.top_k), dtype=torch.int32, device=DEV),
+             "topk_w": torch.empty((T, wl.top_k), dtype=torch.float32, device=DEV)}
+        run_forward(wl, W, x, routing=r)
+        outs.append({k: v.cpu().numpy() for k, v in r.items()})
+    for o in outs[1:]:
+        for k in o:
+            assert np.array_equal(o[k].view(np.uint32), outs[0][k].view(np.uint32)), k

@@ -73,15 +73,21 @@ def run(wl, W, x, y_dtype):
 
 
 def reference(wl, W, x, tokens):
+    """Oracle output for `tokens`, routed as moe_forward routed (its own logits,
+    checked bit for bit against the oracle's selection on them)."""
     cfg = cfg_of(wl)
     T = x.shape[0]
-    logits = torch.empty((T, wl.n_experts), dtype=torch.float32, device=DEV)
-    idx = torch.empty((T, wl.top_k), dtype=torch.int32, device=DEV)
-    w = torch.empty((T, wl.top_k), dtype=torch.float32, device=DEV)
-    moe.moe_route(cfg, x, W["w_router"], logits, W["bias"], idx, w)
+    r = {"logits": torch.empty((T, wl.n_experts), dtype=torch.float32, device=DEV),
+         "topk_idx": torch.empty((T, wl.top_k), dtype=torch.int32, device=DEV),
+         "topk_w": torch.empty((T, wl.top_k), dtype=torch.float32, device=DEV)}
+    ws = torch.empty(moe.workspace_size(cfg, T), dtype=torch.uint8, device=DEV)
+    y = torch.empty((T, wl.d), dtype=torch.float32, device=DEV)
+    moe.moe_forward(cfg, weights_for_forward(W), x, W["bias"], y, workspace=ws, routing_out=r)
     torch.cuda.synchronize()
-    ridx, rw = oracle.select(logits.cpu().numpy(), W["bias"].cpu().numpy(), wl.n_groups, wl.topk_groups, wl.top_k)
-    assert np.array_equal(idx.cpu().numpy(), ridx)
+    ridx, rw = oracle.select(r["logits"].cpu().numpy(), W["bias"].cpu().numpy(), wl.n_groups, wl.topk_groups,
+                             wl.top_k)
+    assert np.array_equal(r["topk_idx"].cpu().numpy(), ridx)
+    assert np.array_equal(r["topk_w"].cpu().numpy().view(np.uint32), rw.view(np.uint32))
     L = oracle_layer(wl, W, np.unique(ridx[tokens]))
     return oracle.expert_tokens(L, x_host(x), ridx, rw, tokens)
 
