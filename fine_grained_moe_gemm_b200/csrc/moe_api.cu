@@ -117,6 +117,7 @@ int pick_bn(long long rows_per_expert) {
 
 constexpr int kBoxRows = 32;  // token rows per B-operand TMA box
 constexpr int kFp8MaxBn = 64;  // FP8 GEMMs hold their promoted sums in registers
+constexpr int kPairBoxRows = 16;  // token rows per B box in the CTA-pair GEMM (each CTA loads half)
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -372,6 +373,10 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     const int ldh = H > Hs ? H : Hs;
     int bn = pick_bn(((long long)T * k + E - 1) / E);
     if (fp8 && bn > kFp8MaxBn) bn = kFp8MaxBn;
+    // wide token tiles run on CTA pairs (2-SM MMA): 256 features per gate/up
+    // item, 512 rows per down item, each SM loading half of the token rows
+    const bool pair = !fp8 && bn == 256 && H % 256 == 0 && Hs % 256 == 0 && d % 512 == 0 && di.sm_count >= 2;
+    const int box_rows = pair ? kPairBoxRows : kBoxRows;
 
     auto mark = [&](int i) {
         if (events && events->ev[i]) cudaEventRecord((cudaEvent_t)events->ev[i], s);
@@ -402,9 +407,9 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     pa.item_off_gu = W.item_gu;
     pa.item_off_dn = W.item_dn;
     pa.bn_gu = pa.bn_dn = bn;
-    pa.mt_gu_routed = H / 128;
-    pa.mt_gu_shared = Hs / 128;
-    pa.mt_dn = (d + 255) / 256;
+    pa.mt_gu_routed = pair ? H / 256 : H / 128;
+    pa.mt_gu_shared = pair ? Hs / 256 : Hs / 128;
+    pa.mt_dn = pair ? d / 512 : (d + 255) / 256;
     if (launch_permute(pa, s) != cudaSuccess) return MOE_ERR_CUDA;
     if (fp8) {
         if (launch_quant_act(static_cast<const __nv_bfloat16*>(x), T, d, W.x_q, W.sx, s) != cudaSuccess ||
@@ -431,15 +436,15 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
         g.s0 = g.a0;
         g.s1 = g.a1;
     }
-    if (!(fp8 ? map_u8(&g.b, W.xq_perm, rows_max, d, kBoxRows) : map_bf16(&g.b, W.x_perm, rows_max, d, kBoxRows)))
+    if (!(fp8 ? map_u8(&g.b, W.xq_perm, rows_max, d, box_rows) : map_bf16(&g.b, W.x_perm, rows_max, d, box_rows)))
         return MOE_ERR_CUDA;
     g.item_off = W.item_gu;
     g.row_off = W.row_off;
     g.n_groups = NG;
     g.n_routed = E;
     g.K_routed = g.K_shared = d;
-    g.mt_routed = H / 128;
-    g.mt_shared = Hs / 128;
+    g.mt_routed = pa.mt_gu_routed;
+    g.mt_shared = pa.mt_gu_shared;
     g.rows_per_expert = H;
     g.h = W.h_perm;
     g.ldh = ldh;
@@ -456,9 +461,10 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
         g.hsT = W.shT;
         g.hs_ld = rows_max;
     }
-    if ((fp8 ? launch_gemm_fp8(MODE_GATEUP, bn, &g, di.sm_count, s) : launch_gemm(MODE_GATEUP, bn, &g, di.sm_count, s)) !=
-        cudaSuccess)
-        return MOE_ERR_CUDA;
+    const cudaError_t egu = fp8    ? launch_gemm_fp8(MODE_GATEUP, bn, &g, di.sm_count, s)
+                            : pair ? launch_gemm2(MODE_GATEUP, &g, di.sm_count, s)
+                                   : launch_gemm(MODE_GATEUP, bn, &g, di.sm_count, s);
+    if (egu != cudaSuccess) return MOE_ERR_CUDA;
     mark(3);
 
     // (5) down GEMM, routing-weight scale and un-permute scatter into fp32
@@ -476,7 +482,7 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     }
     dn.a1 = dn.a0;
     dn.s1 = dn.s0;
-    if (!(fp8 ? map_u8(&dn.b, W.hq, rows_max, ldh, kBoxRows) : map_bf16(&dn.b, W.h_perm, rows_max, ldh, kBoxRows)))
+    if (!(fp8 ? map_u8(&dn.b, W.hq, rows_max, ldh, box_rows) : map_bf16(&dn.b, W.h_perm, rows_max, ldh, box_rows)))
         return MOE_ERR_CUDA;
     dn.item_off = W.item_dn;
     dn.row_off = W.row_off;
@@ -484,7 +490,7 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     dn.n_routed = E;
     dn.K_routed = H;
     dn.K_shared = Hs;
-    dn.mt_routed = dn.mt_shared = (d + 255) / 256;
+    dn.mt_routed = dn.mt_shared = pa.mt_dn;
     dn.rows_per_expert = d;
     dn.y = yacc;
     dn.row_coef = W.row_coef;
@@ -497,9 +503,10 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
         dn.sbT = W.shT;
         dn.sb_ld = rows_max;
     }
-    if ((fp8 ? launch_gemm_fp8(MODE_DOWN, bn, &dn, di.sm_count, s) : launch_gemm(MODE_DOWN, bn, &dn, di.sm_count, s)) !=
-        cudaSuccess)
-        return MOE_ERR_CUDA;
+    const cudaError_t edn = fp8    ? launch_gemm_fp8(MODE_DOWN, bn, &dn, di.sm_count, s)
+                            : pair ? launch_gemm2(MODE_DOWN, &dn, di.sm_count, s)
+                                   : launch_gemm(MODE_DOWN, bn, &dn, di.sm_count, s);
+    if (edn != cudaSuccess) return MOE_ERR_CUDA;
     mark(4);
 
     if (y_dtype == MOE_BF16 &&
