@@ -462,8 +462,11 @@ def main():
     p.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
     p.add_argument("--cpu-sample", type=int, default=0, help="tokens of the oracle sample (0: min(T, 8))")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--tokens", type=int, default=0, help="override the workload's T (sweeps; default: as named)")
     args = p.parse_args()
     wl = WORKLOADS[args.workload]
+    if args.tokens > 0:
+        wl = wl.with_T(args.tokens)
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_ours(args, wl)

@@ -168,7 +168,7 @@ class MoeStageEvents(ctypes.Structure):
 
 
 class MoeRoutingOut(ctypes.Structure):
-    _fields_ = [("logits", ctypes.c_void_p), ("topk_idx", ctypes.c_void_p), ("topk_w", ctypes.c_void_p)]
+    _fields_ = [(n, ctypes.c_void_p) for n in ("logits", "topk_idx", "topk_w", "counts", "offsets", "src", "inv")]
 
 
 STAGES = ("route", "permute+gather", "gate_up", "down+combine", "cast")
@@ -180,7 +180,7 @@ def moe_forward(cfg: MoeConfig, weights, x, bias, y, accumulate: bool = False, w
     least ``workspace_size(cfg, T)`` bytes.  ``stage_events``: optional list of six torch.cuda.Event(
     enable_timing=True) recorded around the stages (see ``STAGES``).  ``routing_out``: optional dict with any of
     ``logits`` [T, E] f32, ``topk_idx`` [T, k] int32, ``topk_w`` [T, k] f32 CUDA tensors that receive the routing
-    the layer used."""
+    the layer used, and ``counts`` [E], ``offsets`` [E+1], ``src``/``inv`` [T*k] int32 for its permutation."""
     for n, t in (("x", x), ("bias", bias), ("y", y), ("workspace", workspace)):
         _dev(t, n)
     mw = weights if isinstance(weights, MoeWeights) else make_weights(weights)
@@ -196,7 +196,7 @@ def moe_forward(cfg: MoeConfig, weights, x, bias, y, accumulate: bool = False, w
     ro = None
     if routing_out is not None:
         ro = MoeRoutingOut()
-        for name in ("logits", "topk_idx", "topk_w"):
+        for name, _ in MoeRoutingOut._fields_:
             t = routing_out.get(name)
             if t is not None:
                 _dev(t, name)

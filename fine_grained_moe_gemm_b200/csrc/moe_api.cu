@@ -117,6 +117,7 @@ int pick_bn(long long rows_per_expert) {
 
 constexpr int kBoxRows = 32;  // token rows per B-operand TMA box
 constexpr int kFp8MaxBn = 64;  // FP8 GEMMs hold their promoted sums in registers
+constexpr int kPermuteMultiMinT = 1024;  // tokens above which the permutation runs on many CTAs
 constexpr int kPairBoxRows = 16;  // token rows per B box in the CTA-pair GEMM (each CTA loads half)
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -148,6 +149,7 @@ bool map_u8(CUtensorMap* m, const void* p, uint64_t rows, uint64_t cols, uint32_
 struct Workspace {
     float* logits;
     float* part;             // split-K partial router logits
+    int32_t* hist;           // per-CTA expert histograms of the multi-CTA permutation
     int32_t* idx;
     float* w;
     int32_t* counts;
@@ -189,6 +191,7 @@ Workspace layout(const moe_config* c, int T, void* base) {
     w.part = (float*)take(router_part_rows(T) * E * 4);
     w.idx = (int32_t*)take((size_t)T * k * 4);
     w.w = (float*)take((size_t)T * k * 4);
+    w.hist = (int32_t*)take((size_t)permute_blocks(T) * E * 4);
     w.counts = (int32_t*)take(E * 4);
     w.offsets = (int32_t*)take((E + 1) * 4);
     w.src = (int32_t*)take((size_t)T * k * 4);
@@ -365,6 +368,15 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
         if (routing->logits) W.logits = routing->logits;
         if (routing->topk_idx) W.idx = routing->topk_idx;
         if (routing->topk_w) W.w = routing->topk_w;
+        if ((routing->counts && (reinterpret_cast<uintptr_t>(routing->counts) & 3u)) ||
+            (routing->offsets && (reinterpret_cast<uintptr_t>(routing->offsets) & 3u)) ||
+            (routing->src && (reinterpret_cast<uintptr_t>(routing->src) & 3u)) ||
+            (routing->inv && (reinterpret_cast<uintptr_t>(routing->inv) & 3u)))
+            return MOE_ERR_INVALID_ARG;
+        if (routing->counts) W.counts = routing->counts;
+        if (routing->offsets) W.offsets = routing->offsets;
+        if (routing->src) W.src = routing->src;
+        if (routing->inv) W.inv = routing->inv;
     }
     const int E = cfg->n_experts, k = cfg->top_k, d = cfg->d, H = cfg->hidden;
     const int Hs = cfg->n_shared ? cfg->shared_hidden : H;
@@ -410,7 +422,9 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     pa.mt_gu_routed = pair ? H / 256 : H / 128;
     pa.mt_gu_shared = pair ? Hs / 256 : Hs / 128;
     pa.mt_dn = pair ? d / 512 : (d + 255) / 256;
-    if (launch_permute(pa, s) != cudaSuccess) return MOE_ERR_CUDA;
+    // a single CTA sorts decode-sized batches in one launch; large batches use many CTAs
+    const cudaError_t ep = T > kPermuteMultiMinT ? launch_permute_multi(pa, W.hist, s) : launch_permute(pa, s);
+    if (ep != cudaSuccess) return MOE_ERR_CUDA;
     if (fp8) {
         if (launch_quant_act(static_cast<const __nv_bfloat16*>(x), T, d, W.x_q, W.sx, s) != cudaSuccess ||
             launch_gather_fp8(W.x_q, W.sx, d, W.row_tok, W.row_off + NG, rows_max, W.xq_perm, W.sxT, di.sm_count,

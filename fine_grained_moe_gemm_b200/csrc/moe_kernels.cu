@@ -304,6 +304,121 @@ __global__ void __launch_bounds__(PERM_THREADS, 1) permute_kernel(PermuteArgs a,
     }
 }
 
+// ---------------------------------------------------------------------------- multi-CTA permutation
+// The same counting sort over many CTAs for large T: each CTA owns
+// PERM_TB consecutive tokens (8 warps x 32).
+//   count:   per-CTA histogram (per-warp lane masks, as above) -> hist[b][e]
+//   scan:    one CTA: hist[b][e] -> exclusive prefix over b (the CTA's base
+//            inside expert e), counts, offsets, group extents, tile schedules
+//   scatter: per CTA, warp bases from the masks, rows = offsets[e] + hist[b][e]
+//            + warp base + rank among the lower lanes
+// The rows come out identical to the single-CTA kernel's (ascending t).
+constexpr int PERM_TB = 256;
+
+__device__ __forceinline__ void build_lane_masks(const PermuteArgs& a, unsigned* s_mask, int t0, bool flag_bad) {
+    const int E = a.E, k = a.k, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int i = tid; i < (PERM_TB / 32) * E; i += PERM_TB) s_mask[i] = 0u;
+    __syncthreads();
+    const int t = t0 + warp * 32 + lane;
+    if (t < a.T) {
+        bool bad = false;
+        for (int j = 0; j < k; ++j) {
+            const int e = a.idx[(size_t)t * k + j];
+            if (e >= 0 && e < E) atomicOr(&s_mask[warp * E + e], 1u << lane);
+            else bad = true;
+        }
+        if (bad && flag_bad) set_dev_error(MOE_DEVERR_BAD_EXPERT);
+    }
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(PERM_TB) permute_count_kernel(PermuteArgs a, int32_t* __restrict__ hist) {
+    extern __shared__ unsigned pcm[];
+    build_lane_masks(a, pcm, blockIdx.x * PERM_TB, true);
+    for (int e = threadIdx.x; e < a.E; e += PERM_TB) {
+        int c = 0;
+        for (int w = 0; w < PERM_TB / 32; ++w) c += __popc(pcm[w * a.E + e]);
+        hist[(size_t)blockIdx.x * a.E + e] = c;
+    }
+}
+
+__global__ void __launch_bounds__(PERM_THREADS, 1) permute_scan_kernel(PermuteArgs a, int32_t* __restrict__ hist,
+                                                                       int nb) {
+    extern __shared__ int psm2[];
+    const int E = a.E, T = a.T, tid = threadIdx.x;
+    int* s_scan = psm2;                      // [PERM_SCAN_CAP]
+    int* s_wsum = s_scan + PERM_SCAN_CAP;    // [64]
+    for (int e = tid; e < E; e += PERM_THREADS) {
+        int run = 0;
+        for (int b = 0; b < nb; ++b) {
+            const int v = hist[(size_t)b * E + e];
+            hist[(size_t)b * E + e] = run;
+            run += v;
+        }
+        a.counts[e] = run;
+        s_scan[e] = run;
+    }
+    __syncthreads();
+    const int tot = block_excl_scan(s_scan, E, s_wsum);
+    for (int e = tid; e < E; e += PERM_THREADS) a.offsets[e] = s_scan[e];
+    if (tid == 0) a.offsets[E] = tot;
+    const int NG = E + a.n_shared;
+    for (int g = tid; g <= NG; g += PERM_THREADS) a.row_off[g] = g <= E ? (g < E ? s_scan[g] : tot) : tot + T;
+    __syncthreads();
+    for (int pass = 0; pass < 2; ++pass) {
+        const int bn = pass == 0 ? a.bn_gu : a.bn_dn;
+        for (int g = tid; g < NG; g += PERM_THREADS) {
+            const int n = g < E ? a.counts[g] : T;
+            const int mt = pass == 0 ? (g < E ? a.mt_gu_routed : a.mt_gu_shared) : a.mt_dn;
+            s_scan[g] = ((n + bn - 1) / bn) * mt;
+        }
+        __syncthreads();
+        const int items = block_excl_scan(s_scan, NG, s_wsum);
+        int32_t* dst = pass == 0 ? a.item_off_gu : a.item_off_dn;
+        for (int g = tid; g < NG; g += PERM_THREADS) dst[g] = s_scan[g];
+        if (tid == 0) dst[NG] = items;
+        __syncthreads();
+    }
+    for (int t = tid; t < T * a.n_shared; t += PERM_THREADS) {
+        a.row_tok[tot + t] = t;
+        a.row_coef[tot + t] = 1.0f;
+    }
+}
+
+__global__ void __launch_bounds__(PERM_TB) permute_scatter_kernel(PermuteArgs a, const int32_t* __restrict__ hist) {
+    extern __shared__ unsigned psc[];
+    const int E = a.E, k = a.k, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    unsigned* s_mask = psc;                                       // [8][E]
+    int* s_wbase = reinterpret_cast<int*>(psc + (PERM_TB / 32) * E);  // [8][E]
+    const int t0 = blockIdx.x * PERM_TB;
+    build_lane_masks(a, s_mask, t0, false);
+    for (int e = tid; e < E; e += PERM_TB) {
+        int acc = a.offsets[e] + hist[(size_t)blockIdx.x * E + e];
+        for (int w = 0; w < PERM_TB / 32; ++w) {
+            s_wbase[w * E + e] = acc;
+            acc += __popc(s_mask[w * E + e]);
+        }
+    }
+    __syncthreads();
+    const int t = t0 + warp * 32 + lane;
+    if (t < a.T) {
+        const unsigned lower = (1u << lane) - 1u;
+        for (int j = 0; j < k; ++j) {
+            const int p = t * k + j;
+            const int e = a.idx[p];
+            if (e >= 0 && e < E) {
+                const int row = s_wbase[warp * E + e] + __popc(s_mask[warp * E + e] & lower);
+                a.src[row] = p;
+                a.inv[p] = row;
+                a.row_tok[row] = t;
+                a.row_coef[row] = a.routed_scale * a.topk_w[p];
+            } else {
+                a.inv[p] = -1;
+            }
+        }
+    }
+}
+
 // ============================================================================ gather
 __global__ void __launch_bounds__(256) gather_rows_kernel(const void* __restrict__ x, int x_f32, int d,
                                                           const int32_t* __restrict__ row_tok,
@@ -569,6 +684,28 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s) {
         attr_set[dev] = true;
     }
     permute_kernel<<<1, PERM_THREADS, smem, s>>>(a, WR);
+    return cudaGetLastError();
+}
+
+int permute_blocks(int T) { return (T + PERM_TB - 1) / PERM_TB; }
+
+cudaError_t launch_permute_multi(const PermuteArgs& a, int32_t* hist, cudaStream_t s) {
+    const int nb = permute_blocks(a.T);
+    const size_t smem_c = (size_t)(PERM_TB / 32) * a.E * 4;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(permute_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             64 * 1024);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    permute_count_kernel<<<nb, PERM_TB, smem_c, s>>>(a, hist);
+    permute_scan_kernel<<<1, PERM_THREADS, (PERM_SCAN_CAP + 64) * 4, s>>>(a, hist, nb);
+    permute_scatter_kernel<<<nb, PERM_TB, 2 * smem_c, s>>>(a, hist);
     return cudaGetLastError();
 }
 

@@ -80,6 +80,9 @@ cudaError_t launch_router_f32(const float* x, const __nv_bfloat16* wr, int T, in
 cudaError_t launch_select(const float* logits, const float* bias, int T, int E, int G, int tg, int k,
                           int32_t* idx, float* w, cudaStream_t s, const float* parts = nullptr, int n_parts = 1);
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
+// Forward mode only, many CTAs: needs hist [permute_blocks(T) * E] int32 of scratch.
+int permute_blocks(int T);
+cudaError_t launch_permute_multi(const PermuteArgs& a, int32_t* hist, cudaStream_t s);
 // x_perm[r, :] = x[row_tok[r], :] (fp32 input rounded to bf16) for r < row_off[n_groups]
 cudaError_t launch_gather(const void* x, bool x_f32, int d, const int32_t* row_tok, const int32_t* n_rows_dev,
                           int max_rows, __nv_bfloat16* x_perm, int n_sm, cudaStream_t s);

@@ -184,15 +184,21 @@ typedef struct {
     moe_event_t ev[6];
 } moe_stage_events;
 
-/* Optional outputs of moe_forward_ex: the routing the layer used.  Each
- * non-NULL pointer is a caller device buffer that receives the router logits
- * [T, E] fp32, topk_idx [T, k] int32 or topk_w [T, k] fp32 (unscaled) exactly
- * as the layer computed and consumed them.  (moe_route runs the router
- * without splitting K, so its logits may differ from these in the last bits.) */
+/* Optional outputs of moe_forward_ex: the routing and permutation the layer
+ * used.  Each non-NULL pointer is a caller device buffer that receives, exactly
+ * as the layer computed and consumed them: the router logits [T, E] fp32,
+ * topk_idx [T, k] int32, topk_w [T, k] fp32 (unscaled), and the permutation
+ * counts [E], offsets [E+1], src [T*k], inv [T*k] int32 as moe_permute defines
+ * them.  (moe_route runs the router without splitting K, so its logits may
+ * differ from these in the last bits.) */
 typedef struct {
     float* logits;
     int32_t* topk_idx;
     float* topk_w;
+    int32_t* counts;
+    int32_t* offsets;
+    int32_t* src;
+    int32_t* inv;
 } moe_routing_out;
 
 /* moe_forward, recording the stage events when `events` is not NULL and

@@ -52,14 +52,22 @@ def forward_routing(wl, W, x):
     the oracle's selection on those logits, and its logits against the oracle's
     fp64 router within tolerance."""
     T = x.shape[0]
-    r = {"logits": torch.empty((T, wl.n_experts), dtype=torch.float32, device=DEV),
-         "topk_idx": torch.empty((T, wl.top_k), dtype=torch.int32, device=DEV),
-         "topk_w": torch.empty((T, wl.top_k), dtype=torch.float32, device=DEV)}
+    E, k = wl.n_experts, wl.top_k
+    r = {"logits": torch.empty((T, E), dtype=torch.float32, device=DEV),
+         "topk_idx": torch.empty((T, k), dtype=torch.int32, device=DEV),
+         "topk_w": torch.empty((T, k), dtype=torch.float32, device=DEV),
+         "counts": torch.empty(E, dtype=torch.int32, device=DEV),
+         "offsets": torch.empty(E + 1, dtype=torch.int32, device=DEV),
+         "src": torch.empty(T * k, dtype=torch.int32, device=DEV),
+         "inv": torch.empty(T * k, dtype=torch.int32, device=DEV)}
     run_forward(wl, W, x, routing=r)
     l = r["logits"].cpu().numpy()
     ridx, rw = oracle.select(l, W["bias"].cpu().numpy(), wl.n_groups, wl.topk_groups, wl.top_k)
     assert np.array_equal(r["topk_idx"].cpu().numpy(), ridx)
     assert np.array_equal(r["topk_w"].cpu().numpy().view(np.uint32), rw.view(np.uint32))
+    # the layer's own permutation (single- or multi-CTA), bit-exact
+    for got, ref in zip((r["counts"], r["offsets"], r["src"], r["inv"]), oracle.permute(ridx, E)):
+        assert np.array_equal(got.cpu().numpy(), ref)
     rows = np.unique(np.linspace(0, T - 1, min(T, 16)).astype(np.int64))
     l_ref = oracle.router_logits(x_host(x[torch.from_numpy(rows).to(DEV)]), u16(W["w_router"]))
     rms = float(np.sqrt(np.mean(l_ref.astype(np.float64) ** 2)))
