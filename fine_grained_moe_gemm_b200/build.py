@@ -9,7 +9,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmoe_b200.so")
 SOURCES = ["moe_kernels.cu", "moe_api.cu", "moe_noalloc.cu"]
-HEADERS = ["moe_device.cuh", "moe_gemm.cuh", "moe_gemm_fp8.cuh", "moe_gemm2.cuh", "moe_launch.h", os.path.join("..", "..", "include", "moe.h")]
+HEADERS = ["moe_device.cuh", "moe_gemm.cuh", "moe_gemm_fp8.cuh", "moe_gemm2.cuh", "moe_gemm2_fp8.cuh", "moe_launch.h", os.path.join("..", "..", "include", "moe.h")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

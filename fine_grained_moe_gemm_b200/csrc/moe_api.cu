@@ -384,11 +384,15 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     const int rows_max = T * k + cfg->n_shared * T;
     const int ldh = H > Hs ? H : Hs;
     int bn = pick_bn(((long long)T * k + E - 1) / E);
-    if (fp8 && bn > kFp8MaxBn) bn = kFp8MaxBn;
-    // wide token tiles run on CTA pairs (2-SM MMA): 256 features per gate/up
-    // item, 512 rows per down item, each SM loading half of the token rows
+    // wide token tiles run on CTA pairs (2-SM MMA), each SM loading half of the
+    // token rows.  bf16: 256 rows per item, 256 features per gate/up item, 512
+    // rows per down item.  FP8: 128 rows per item (the promoted sums live in
+    // registers), 128 features per gate/up item, 256 rows per down item.
     const bool pair = !fp8 && bn == 256 && H % 256 == 0 && Hs % 256 == 0 && d % 512 == 0 && di.sm_count >= 2;
-    const int box_rows = pair ? kPairBoxRows : kBoxRows;
+    const bool pair8 = fp8 && bn >= 128 && di.sm_count >= 2;
+    if (pair8) bn = 128;
+    else if (fp8 && bn > kFp8MaxBn) bn = kFp8MaxBn;
+    const int box_rows = (pair || pair8) ? kPairBoxRows : kBoxRows;
 
     auto mark = [&](int i) {
         if (events && events->ev[i]) cudaEventRecord((cudaEvent_t)events->ev[i], s);
@@ -421,7 +425,7 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     pa.bn_gu = pa.bn_dn = bn;
     pa.mt_gu_routed = pair ? H / 256 : H / 128;
     pa.mt_gu_shared = pair ? Hs / 256 : Hs / 128;
-    pa.mt_dn = pair ? d / 512 : (d + 255) / 256;
+    pa.mt_dn = pair ? d / 512 : (d + 255) / 256;  // pair8: 256 down rows per item, as the 1-CTA kernels
     // a single CTA sorts decode-sized batches in one launch; large batches use many CTAs
     const cudaError_t ep = T > kPermuteMultiMinT ? launch_permute_multi(pa, W.hist, s) : launch_permute(pa, s);
     if (ep != cudaSuccess) return MOE_ERR_CUDA;
@@ -442,10 +446,12 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     };
     GemmArgs g;
     memset(&g, 0, sizeof(g));
-    if (!wmap(&g.a0, wt->w_gate, (uint64_t)E * H, d, 128) || !wmap(&g.a1, wt->w_up, (uint64_t)E * H, d, 128))
+    // weight rows per TMA box: the FP8 pair kernel stacks 64 gate over 64 up rows per CTA
+    const uint32_t gu_box = pair8 ? 64 : 128;
+    if (!wmap(&g.a0, wt->w_gate, (uint64_t)E * H, d, gu_box) || !wmap(&g.a1, wt->w_up, (uint64_t)E * H, d, gu_box))
         return MOE_ERR_CUDA;
     if (cfg->n_shared) {
-        if (!wmap(&g.s0, wt->ws_gate, Hs, d, 128) || !wmap(&g.s1, wt->ws_up, Hs, d, 128)) return MOE_ERR_CUDA;
+        if (!wmap(&g.s0, wt->ws_gate, Hs, d, gu_box) || !wmap(&g.s1, wt->ws_up, Hs, d, gu_box)) return MOE_ERR_CUDA;
     } else {
         g.s0 = g.a0;
         g.s1 = g.a1;
@@ -475,7 +481,8 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
         g.hsT = W.shT;
         g.hs_ld = rows_max;
     }
-    const cudaError_t egu = fp8    ? launch_gemm_fp8(MODE_GATEUP, bn, &g, di.sm_count, s)
+    const cudaError_t egu = pair8  ? launch_gemm2_fp8(MODE_GATEUP, &g, di.sm_count, s)
+                            : fp8  ? launch_gemm_fp8(MODE_GATEUP, bn, &g, di.sm_count, s)
                             : pair ? launch_gemm2(MODE_GATEUP, &g, di.sm_count, s)
                                    : launch_gemm(MODE_GATEUP, bn, &g, di.sm_count, s);
     if (egu != cudaSuccess) return MOE_ERR_CUDA;
@@ -517,7 +524,8 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
         dn.sbT = W.shT;
         dn.sb_ld = rows_max;
     }
-    const cudaError_t edn = fp8    ? launch_gemm_fp8(MODE_DOWN, bn, &dn, di.sm_count, s)
+    const cudaError_t edn = pair8  ? launch_gemm2_fp8(MODE_DOWN, &dn, di.sm_count, s)
+                            : fp8  ? launch_gemm_fp8(MODE_DOWN, bn, &dn, di.sm_count, s)
                             : pair ? launch_gemm2(MODE_DOWN, &dn, di.sm_count, s)
                                    : launch_gemm(MODE_DOWN, bn, &dn, di.sm_count, s);
     if (edn != cudaSuccess) return MOE_ERR_CUDA;

@@ -95,7 +95,16 @@ __device__ __forceinline__ void mma2_commit_local(uint64_t* bar) {
                  : "memory");
 }
 
+// Arrive on an mbarrier of either CTA of the pair (shared::cluster address).
+// Used to hand TMEM back to the MMA issuer after tcgen05.fence::before_thread_sync;
+// no data other than TMEM is published, so no cluster-scope release is needed.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+
+// Arrive with release at cluster scope: the peer's acquire-wait then sees this
+// thread's earlier stores to its shared memory.
+__device__ __forceinline__ void mbar_arrive_cluster_release(uint32_t bar_cluster) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 

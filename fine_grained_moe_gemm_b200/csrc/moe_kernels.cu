@@ -17,6 +17,7 @@
 #include "moe_gemm.cuh"
 #include "moe_gemm_fp8.cuh"
 #include "moe_gemm2.cuh"
+#include "moe_gemm2_fp8.cuh"
 #include "moe_launch.h"
 
 namespace moe {
@@ -628,6 +629,29 @@ cudaError_t launch_gemm2(int mode, const GemmArgs* args, int grid, cudaStream_t 
     if (grid < 2) return cudaErrorInvalidValue;
     if (mode == MODE_GATEUP) return launch_gemm2_t<GEMM_GATEUP>(args, grid, s);
     if (mode == MODE_DOWN) return launch_gemm2_t<GEMM_DOWN>(args, grid, s);
+    return cudaErrorInvalidValue;
+}
+
+template <int MODE>
+static cudaError_t launch_gemm2_fp8_t(const GemmArgs* args, int grid, cudaStream_t s) {
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(moe_gemm2_fp8_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             Gemm2Fp8Cfg::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    moe_gemm2_fp8_kernel<MODE><<<grid, GEMM_THREADS, Gemm2Fp8Cfg::SMEM_BYTES, s>>>(*args);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm2_fp8(int mode, const GemmArgs* args, int grid, cudaStream_t s) {
+    grid &= ~1;
+    if (grid < 2) return cudaErrorInvalidValue;
+    if (mode == MODE_GATEUP) return launch_gemm2_fp8_t<GEMM_GATEUP>(args, grid, s);
+    if (mode == MODE_DOWN) return launch_gemm2_fp8_t<GEMM_DOWN>(args, grid, s);
     return cudaErrorInvalidValue;
 }
 

@@ -95,6 +95,8 @@ cudaError_t launch_gather_fp8(const uint8_t* xq, const float* sx, int d, const i
 int gemm_fp8_smem_bytes(int mode, int bn);
 // CTA-pair (2-SM MMA) bf16 grouped GEMM, 256 token rows per item; grid even.
 cudaError_t launch_gemm2(int mode, const GemmArgs* args, int grid, cudaStream_t s);
+// CTA-pair FP8 grouped GEMM, 128 token rows per item; grid even.
+cudaError_t launch_gemm2_fp8(int mode, const GemmArgs* args, int grid, cudaStream_t s);
 cudaError_t launch_gemm_fp8(int mode, int bn, const GemmArgs* args, int grid, cudaStream_t s);
 // y[i] = bf16(acc[i] (+ y[i]))
 cudaError_t launch_finalize_bf16(const float* acc, __nv_bfloat16* y, size_t n, bool accumulate, cudaStream_t s);
