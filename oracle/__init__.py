@@ -73,6 +73,7 @@ def lib():
             L.orc_permute.restype = ctypes.c_int
             L.orc_permute.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P]
             L.orc_quant_act.argtypes = [P, ctypes.c_int, ctypes.c_int, P, P]
+            L.orc_update_bias.argtypes = [P, ctypes.c_int, P, ctypes.c_float]
             L.orc_expert_tokens.restype = ctypes.c_int
             L.orc_expert_tokens.argtypes = [ctypes.POINTER(OrcLayer), P, P, P, P, ctypes.c_int, ctypes.c_int, P]
             L.orc_expert_single.argtypes = [ctypes.POINTER(OrcLayer), ctypes.c_int, P, P]
@@ -162,6 +163,15 @@ def permute(idx: np.ndarray, n_experts: int):
     if rc != 0:
         raise ValueError("oracle permute: expert id out of range")
     return counts, offsets, src, inv
+
+
+def update_bias(counts: np.ndarray, bias: np.ndarray, gamma: float = 1e-3) -> np.ndarray:
+    """Bias controller ("MoE router" box, update_bias): a new fp32 bias, -gamma for
+    experts above the mean count, +gamma for the others."""
+    c = np.ascontiguousarray(counts, dtype=np.int32)
+    b = np.ascontiguousarray(bias, dtype=np.float32).copy()
+    lib().orc_update_bias(_ptr(c), c.size, _ptr(b), float(np.float32(gamma)))
+    return b
 
 
 def quant_act(x_bf16: np.ndarray):

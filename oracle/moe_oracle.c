@@ -294,6 +294,25 @@ int orc_permute(const int32_t* idx, int T, int k, int E, int32_t* counts,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Bias controller ("MoE router" box, update_bias; teardown section 6: the   */
+/* bias is lowered for overloaded experts and raised for underloaded ones    */
+/* after each step):                                                         */
+/*   mean = (sum of counts) / E                     (fp32, as counts.mean()) */
+/*   bias[e] -= gamma  if counts[e] > mean   else  bias[e] += gamma  (fp32)   */
+/* ------------------------------------------------------------------------ */
+
+void orc_update_bias(const int32_t* counts, int E, float* bias, float gamma)
+{
+    int64_t sum = 0;
+    for (int e = 0; e < E; ++e) sum += counts[e];
+    float mean = (float)sum / (float)E;
+    for (int e = 0; e < E; ++e) {
+        if ((float)counts[e] > mean) bias[e] = bias[e] - gamma;
+        else bias[e] = bias[e] + gamma;
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* S6  activation quantisation (teardown, section 10: activations scaled in  */
 /* 1x128 tiles, E4M3).  Per token and 128-channel block, in fp32:            */
 /*   sx = amax / 448 (1 when amax = 0);  q = e4m3_rn_sat(x / sx).            */
