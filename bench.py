@@ -29,8 +29,6 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE-layer tokens/sec (T=128 decode, T=4096 prefill); % of HBM/tensor roofline"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_STEP = 7  # router, select, permute, gather, gate/up GEMM, down GEMM, cast
-KERNELS_PER_STEP_FP8 = 8  # + the activation quantisation
 
 # DRAM traffic of the dominant kernel per launch, from one ncu capture, keyed by
 # workload; valid only while the kernel sources hash to the recorded value.
@@ -337,12 +335,18 @@ def run_ours(args, wl):
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
+    n_launch0 = moe.launch_count()
     with ClockSampler(local) as clk:
         t_start.record(stream)
         for i in range(args.steps):
             step(evs[i])
         t_end.record(stream)
         torch.cuda.synchronize()
+    launches = moe.launch_count() - n_launch0
+    plan = moe.forward_plan(cfg, T)
+    if launches != plan["launches"] * args.steps:
+        raise RuntimeError(f"{launches} kernel launches in the timed region, the plan says "
+                           f"{plan['launches']} per step")
     barrier()
     ms = t_start.elapsed_time(t_end)
     stage_ms = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
@@ -402,7 +406,8 @@ def run_ours(args, wl):
         kr = roofline(kF, kB, stage_ms[k_name] / 1e3, peaks, peak_kind, fp8=wl.fp8)
         tr = NCU_TRAFFIC.get(wl.name)
         kr["traffic"] = tr[0] if tr and tr[1] == kernel_source_hash() else None
-        kr["kernel"] = "moe_gemm_kernel<GATEUP>" if k_name == "gate_up" else "moe_gemm_kernel<DOWN>"
+        kr["kernel"] = ("moe_gemm2" if plan["cta_pair"] else "moe_gemm") + ("_fp8" if plan["fp8"] else "") + \
+            "_kernel<" + ("GATEUP" if k_name == "gate_up" else "DOWN") + ", BN=" + str(plan["token_tile"]) + ">"
         lr = roofline(F, B, step_s, peaks, peak_kind, fp8=wl.fp8)
         # the router GEMM stays bf16 in the FP8 layer
         F_router = 2 * T * wl.n_experts * wl.d
@@ -430,7 +435,8 @@ def run_ours(args, wl):
             "e2e": {"value": round(world * T * e2e_steps / (e2e_ms / 1e3), 1), "unit": UNIT,
                     "h2d_bytes_per_step": x.numel() * x.element_size(),
                     "d2h_bytes_per_step": y.numel() * y.element_size()},
-            "gpu_launches": (KERNELS_PER_STEP_FP8 if wl.fp8 else KERNELS_PER_STEP) * args.steps,
+            "gpu_launches": launches,
+            "plan": plan,
             "clocks": clk.summary(),
             "kernel_source": kernel_source_hash(),
         }

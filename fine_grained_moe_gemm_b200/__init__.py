@@ -77,6 +77,12 @@ def lib():
             L.moe_forward_ex.restype = I
             L.moe_forward_ex.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, I, P, I, I, P,
                                          ctypes.c_size_t, P, P, P]
+            L.moe_forward_plan.restype = I
+            L.moe_forward_plan.argtypes = [ctypes.POINTER(MoeConfig), I, I, ctypes.c_void_p]
+            L.moe_launch_count.restype = ctypes.c_ulonglong
+            L.moe_launch_count.argtypes = []
+            L.moe_update_bias.restype = I
+            L.moe_update_bias.argtypes = [ctypes.POINTER(MoeConfig), P, P, ctypes.c_float, P]
             L.moe_quantize_act.restype = I
             L.moe_quantize_act.argtypes = [P, I, I, P, P, P]
             L.moe_device_error.restype = I
@@ -171,7 +177,20 @@ class MoeRoutingOut(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("logits", "topk_idx", "topk_w", "counts", "offsets", "src", "inv")]
 
 
+class MoePlan(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("token_tile", "cta_pair", "fp8", "router_splits", "permute_ctas",
+                                            "launches")]
+
+
 STAGES = ("route", "permute+gather", "gate_up", "down+combine", "cast")
+
+
+def forward_plan(cfg: MoeConfig, T: int, y_dtype=torch.bfloat16) -> dict:
+    """The kernels ``moe_forward`` runs for ``T`` tokens on the current device (see ``MoePlan``)."""
+    plan = MoePlan()
+    code = MOE_F32 if y_dtype == torch.float32 else MOE_BF16
+    _check(lib().moe_forward_plan(ctypes.byref(cfg), int(T), code, ctypes.byref(plan)), "moe_forward_plan")
+    return {n: getattr(plan, n) for n, _ in MoePlan._fields_}
 
 
 def moe_forward(cfg: MoeConfig, weights, x, bias, y, accumulate: bool = False, workspace=None, stream=None,
@@ -205,6 +224,19 @@ def moe_forward(cfg: MoeConfig, weights, x, bias, y, accumulate: bool = False, w
                                 1 if accumulate else 0, _p(workspace), ws_bytes, _stream(stream),
                                 ctypes.byref(ev) if ev is not None else None,
                                 ctypes.byref(ro) if ro is not None else None), "moe_forward")
+
+
+def launch_count() -> int:
+    """Kernels the library has launched in this process (all devices and streams)."""
+    return int(lib().moe_launch_count())
+
+
+def moe_update_bias(cfg: MoeConfig, counts, bias, gamma: float = 1e-3, stream=None):
+    """Bias controller: bias[e] -= gamma where counts[e] is above the mean count, else += gamma (in place)."""
+    for n, t in (("counts", counts), ("bias", bias)):
+        _dev(t, n)
+    _check(lib().moe_update_bias(ctypes.byref(cfg), _p(counts), _p(bias), float(gamma), _stream(stream)),
+           "moe_update_bias")
 
 
 def moe_quantize_act(x, q, sx, stream=None):

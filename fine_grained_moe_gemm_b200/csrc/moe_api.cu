@@ -219,12 +219,47 @@ Workspace layout(const moe_config* c, int T, void* base) {
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+// The kernels one forward call runs, decided from the shapes and the SM count.
+struct Plan {
+    int bn;              // token rows per grouped-GEMM tile
+    bool fp8;            // e4m3 expert weights
+    bool pair;           // bf16 grouped GEMMs on CTA pairs
+    bool pair8;          // e4m3 grouped GEMMs on CTA pairs
+    int router_parts;    // K splits of the router GEMM (1 with fp32 activations)
+    bool permute_multi;  // many-CTA permutation
+};
+
+Plan make_plan(const moe_config* c, int T, int n_sm) {
+    Plan p;
+    p.fp8 = c->weight_dtype == MOE_E4M3;
+    const int H = c->hidden, Hs = c->n_shared ? c->shared_hidden : c->hidden, d = c->d;
+    p.bn = pick_bn(((long long)T * c->top_k + c->n_experts - 1) / c->n_experts);
+    // wide token tiles run on CTA pairs (2-SM MMA), each SM loading half of the
+    // token rows.  bf16: 256 rows per item, 256 features per gate/up item, 512
+    // rows per down item.  FP8: 128 rows per item (the promoted sums live in
+    // registers), 128 features per gate/up item, 256 rows per down item.
+    p.pair = !p.fp8 && p.bn == 256 && H % 256 == 0 && Hs % 256 == 0 && d % 512 == 0 && n_sm >= 2;
+    p.pair8 = p.fp8 && p.bn >= 128 && n_sm >= 2;
+    if (p.pair8) p.bn = 128;
+    else if (p.fp8 && p.bn > kFp8MaxBn) p.bn = kFp8MaxBn;
+    p.router_parts = 1;
+    if (c->act_dtype != MOE_F32 && c->n_experts <= 256) {
+        p.router_parts = router_splits(T, n_sm);
+        if (p.router_parts > d / 64) p.router_parts = d / 64;  // every split owns at least one K block
+    }
+    // a single CTA sorts decode-sized batches in one launch; large batches use many CTAs
+    p.permute_multi = T > kPermuteMultiMinT;
+    return p;
+}
+
 // Router logits on tensor cores (bf16 x) or CUDA cores (fp32 x), then selection.
 moe_status route_impl(const moe_config* c, const DevInfo& di, const void* x, const void* w_router, float* logits,
-                      const float* bias, int T, int32_t* idx, float* w, cudaStream_t s, float* part = nullptr) {
-    int n_parts = 1;
+                      const float* bias, int T, int32_t* idx, float* w, cudaStream_t s, float* part = nullptr,
+                      int n_parts = 1) {
+    if (!part) n_parts = 1;
     if (x) {
         if (c->act_dtype == MOE_F32) {
+            n_parts = 1;
             cudaError_t e = launch_router_f32(static_cast<const float*>(x),
                                               static_cast<const __nv_bfloat16*>(w_router), T, c->d, c->n_experts,
                                               logits, s);
@@ -233,8 +268,6 @@ moe_status route_impl(const moe_config* c, const DevInfo& di, const void* x, con
             GemmArgs a;
             memset(&a, 0, sizeof(a));
             const int bn = router_bn(T);
-            if (part && c->n_experts <= 256) n_parts = router_splits(T, di.sm_count);
-            if (n_parts > c->d / 64) n_parts = c->d / 64;  // every split owns at least one K block
             if (!map_bf16(&a.a0, w_router, c->n_experts, c->d, 128)) return MOE_ERR_CUDA;
             a.a1 = a.s0 = a.s1 = a.a0;
             if (!map_bf16(&a.b, x, T, c->d, kBoxRows)) return MOE_ERR_CUDA;
@@ -300,6 +333,37 @@ moe_status moe_quantize_act(const void* x, int T, int d, uint8_t* q, float* sx, 
     moe_status st = check_device(&di);
     if (st != MOE_OK) return st;
     return cuda_status(launch_quant_act(static_cast<const __nv_bfloat16*>(x), T, d, q, sx, (cudaStream_t)stream));
+}
+
+unsigned long long moe_launch_count(void) { return launch_count(); }
+
+moe_status moe_forward_plan(const moe_config* cfg, int T, moe_dtype y_dtype, moe_plan* out) {
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (!out || T < 0 || (y_dtype != MOE_F32 && y_dtype != MOE_BF16)) return MOE_ERR_INVALID_ARG;
+    DevInfo di;
+    if ((st = check_device(&di)) != MOE_OK) return st;
+    memset(out, 0, sizeof(*out));
+    if (T == 0) return MOE_OK;
+    const Plan p = make_plan(cfg, T, di.sm_count);
+    out->token_tile = p.bn;
+    out->cta_pair = (p.pair || p.pair8) ? 1 : 0;
+    out->fp8 = p.fp8 ? 1 : 0;
+    out->router_splits = p.router_parts;
+    out->permute_ctas = p.permute_multi ? permute_blocks(T) : 1;
+    // router + selection, permutation, gather (+ quantisation), two GEMMs, bf16 cast
+    out->launches = 2 + (p.permute_multi ? 3 : 1) + (p.fp8 ? 2 : 1) + 2 + (y_dtype == MOE_BF16 ? 1 : 0);
+    return MOE_OK;
+}
+
+moe_status moe_update_bias(const moe_config* cfg, const int32_t* counts, float* bias, float gamma,
+                           moe_stream_t stream) {
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (!counts || !bias || !(gamma == gamma)) return MOE_ERR_INVALID_ARG;
+    DevInfo di;
+    if ((st = check_device(&di)) != MOE_OK) return st;
+    return cuda_status(launch_update_bias(counts, cfg->n_experts, bias, gamma, (cudaStream_t)stream));
 }
 
 moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, int T, int32_t* counts, int32_t* offsets,
@@ -383,15 +447,9 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     const int NG = E + cfg->n_shared;
     const int rows_max = T * k + cfg->n_shared * T;
     const int ldh = H > Hs ? H : Hs;
-    int bn = pick_bn(((long long)T * k + E - 1) / E);
-    // wide token tiles run on CTA pairs (2-SM MMA), each SM loading half of the
-    // token rows.  bf16: 256 rows per item, 256 features per gate/up item, 512
-    // rows per down item.  FP8: 128 rows per item (the promoted sums live in
-    // registers), 128 features per gate/up item, 256 rows per down item.
-    const bool pair = !fp8 && bn == 256 && H % 256 == 0 && Hs % 256 == 0 && d % 512 == 0 && di.sm_count >= 2;
-    const bool pair8 = fp8 && bn >= 128 && di.sm_count >= 2;
-    if (pair8) bn = 128;
-    else if (fp8 && bn > kFp8MaxBn) bn = kFp8MaxBn;
+    const Plan plan = make_plan(cfg, T, di.sm_count);
+    const int bn = plan.bn;
+    const bool pair = plan.pair, pair8 = plan.pair8;
     const int box_rows = (pair || pair8) ? kPairBoxRows : kBoxRows;
 
     auto mark = [&](int i) {
@@ -399,7 +457,7 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     };
     // (1)+(2) router and selection
     mark(0);
-    st = route_impl(cfg, di, x, wt->w_router, W.logits, bias, T, W.idx, W.w, s, W.part);
+    st = route_impl(cfg, di, x, wt->w_router, W.logits, bias, T, W.idx, W.w, s, W.part, plan.router_parts);
     if (st != MOE_OK) return st;
     mark(1);
 
@@ -426,8 +484,7 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     pa.mt_gu_routed = pair ? H / 256 : H / 128;
     pa.mt_gu_shared = pair ? Hs / 256 : Hs / 128;
     pa.mt_dn = pair ? d / 512 : (d + 255) / 256;  // pair8: 256 down rows per item, as the 1-CTA kernels
-    // a single CTA sorts decode-sized batches in one launch; large batches use many CTAs
-    const cudaError_t ep = T > kPermuteMultiMinT ? launch_permute_multi(pa, W.hist, s) : launch_permute(pa, s);
+    const cudaError_t ep = plan.permute_multi ? launch_permute_multi(pa, W.hist, s) : launch_permute(pa, s);
     if (ep != cudaSuccess) return MOE_ERR_CUDA;
     if (fp8) {
         if (launch_quant_act(static_cast<const __nv_bfloat16*>(x), T, d, W.x_q, W.sx, s) != cudaSuccess ||

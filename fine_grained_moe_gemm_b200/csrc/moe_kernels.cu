@@ -1,17 +1,26 @@
 // Kernels of the MoE layer forward pass (sm_100a) and their launchers.
 //
-//   router_f32_kernel   fp32-activation router logits (CUDA cores)
-//   select_kernel       sigmoid, selection bias, group-limited top-k, weights
-//   permute_kernel      histogram / prefix sum / stable scatter by expert, and
-//                       the tile schedules of the grouped GEMMs
-//   gather_rows_kernel  x_perm = x[row_tok] (bf16)
-//   moe_gemm_kernel     tcgen05 grouped GEMM (moe_gemm.cuh)
-//   finalize_kernel     fp32 combine buffer -> bf16 output (+ residual)
+//   router_f32_kernel     fp32-activation router logits (CUDA cores)
+//   select_kernel         sigmoid, selection bias, group-limited top-k, weights
+//   permute_kernel        histogram / prefix sum / stable scatter by expert, and
+//                         the tile schedules of the grouped GEMMs (one CTA);
+//   permute_count/scan/scatter_kernel   the same over many CTAs (large T)
+//   gather_rows_kernel    x_perm = x[row_tok] (bf16)
+//   quant_act_kernel      1x128 e4m3 activation quantisation
+//   gather_fp8_kernel     x_q / scales gathered into expert order
+//   moe_gemm_kernel       tcgen05 grouped GEMM, one CTA per tile (moe_gemm.cuh)
+//   moe_gemm_fp8_kernel   the same for e4m3 with block scales (moe_gemm_fp8.cuh)
+//   moe_gemm2_kernel      CTA-pair grouped GEMM, cta_group::2 (moe_gemm2.cuh)
+//   moe_gemm2_fp8_kernel  CTA-pair e4m3 GEMM (moe_gemm2_fp8.cuh)
+//   update_bias_kernel    selection-bias controller step
+//   finalize_kernel       fp32 combine buffer -> bf16 output (+ residual)
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
+
+#include <atomic>
 
 #include "moe_device.cuh"
 #include "moe_gemm.cuh"
@@ -21,6 +30,11 @@
 #include "moe_launch.h"
 
 namespace moe {
+
+// Kernels launched by this library in this process (all devices and streams).
+static std::atomic<unsigned long long> g_launch_count{0};
+static inline void note_launch() { g_launch_count.fetch_add(1, std::memory_order_relaxed); }
+unsigned long long launch_count() { return g_launch_count.load(std::memory_order_relaxed); }
 
 // ============================================================================ router (fp32 x)
 // logits[t, e] = sum_c x[t, c] * Wr[e, c], fp32 products and fp32 sums
@@ -487,6 +501,30 @@ __global__ void __launch_bounds__(256) gather_fp8_kernel(const uint8_t* __restri
     }
 }
 
+// ============================================================================ bias controller
+// "MoE router" box, update_bias: mean = sum(counts) / E in fp32; experts above
+// it get bias - gamma, the others bias + gamma (one correctly rounded fp32 op).
+__global__ void __launch_bounds__(1024) update_bias_kernel(const int32_t* __restrict__ counts, int E,
+                                                           float* __restrict__ bias, float gamma) {
+    __shared__ long long s_part[32];
+    long long sum = 0;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) sum += counts[e];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = sum;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        long long v = threadIdx.x < (blockDim.x + 31) / 32 ? s_part[threadIdx.x] : 0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (threadIdx.x == 0) s_part[0] = v;
+    }
+    __syncthreads();
+    const float mean = __fdiv_rn(__ll2float_rn(s_part[0]), __int2float_rn(E));
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+        bias[e] = __int2float_rn(counts[e]) > mean ? __fsub_rn(bias[e], gamma) : __fadd_rn(bias[e], gamma);
+}
+
 // ============================================================================ finalize
 __global__ void __launch_bounds__(256) finalize_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ y,
                                                        size_t n8, int accumulate) {
@@ -530,6 +568,7 @@ static cudaError_t launch_gemm_t(const GemmArgs* args, int grid, cudaStream_t s)
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
+    note_launch();
     moe_gemm_kernel<MODE, BN><<<grid, GEMM_THREADS, C::SMEM_BYTES, s>>>(*args);
     return cudaGetLastError();
 }
@@ -580,6 +619,7 @@ static cudaError_t launch_gemm_fp8_t(const GemmArgs* args, int grid, cudaStream_
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
+    note_launch();
     moe_gemm_fp8_kernel<MODE, BN><<<grid, GEMM_THREADS, C::SMEM_BYTES, s>>>(*args);
     return cudaGetLastError();
 }
@@ -620,6 +660,7 @@ static cudaError_t launch_gemm2_t(const GemmArgs* args, int grid, cudaStream_t s
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
+    note_launch();
     moe_gemm2_kernel<MODE><<<grid, GEMM_THREADS, Gemm2Cfg::SMEM_BYTES, s>>>(*args);
     return cudaGetLastError();
 }
@@ -643,6 +684,7 @@ static cudaError_t launch_gemm2_fp8_t(const GemmArgs* args, int grid, cudaStream
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
+    note_launch();
     moe_gemm2_fp8_kernel<MODE><<<grid, GEMM_THREADS, Gemm2Fp8Cfg::SMEM_BYTES, s>>>(*args);
     return cudaGetLastError();
 }
@@ -658,6 +700,7 @@ cudaError_t launch_gemm2_fp8(int mode, const GemmArgs* args, int grid, cudaStrea
 cudaError_t launch_quant_act(const __nv_bfloat16* x, int T, int d, uint8_t* q, float* sx, cudaStream_t s) {
     const long long warps = (long long)T * (d / 128);
     const long long blocks = (warps + 7) / 8;
+    note_launch();
     quant_act_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, T, d, q, sx);
     return cudaGetLastError();
 }
@@ -667,12 +710,14 @@ cudaError_t launch_gather_fp8(const uint8_t* xq, const float* sx, int d, const i
                               cudaStream_t s) {
     int grid = max_rows < n_sm * 8 ? max_rows : n_sm * 8;
     if (grid < 1) grid = 1;
+    note_launch();
     gather_fp8_kernel<<<grid, 256, 0, s>>>(xq, sx, d, row_tok, n_rows_dev, max_rows, xpq, sxT);
     return cudaGetLastError();
 }
 
 cudaError_t launch_router_f32(const float* x, const __nv_bfloat16* wr, int T, int d, int E, float* logits,
                               cudaStream_t s) {
+    note_launch();
     router_f32_kernel<<<T, 256, 0, s>>>(x, wr, T, d, E, logits);
     return cudaGetLastError();
 }
@@ -690,6 +735,7 @@ cudaError_t launch_select(const float* logits, const float* bias, int T, int E, 
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
+    note_launch();
     select_kernel<<<blocks, SELECT_WARPS * 32, smem, s>>>(logits, bias, T, E, G, tg, k, idx, w,
                                                          n_parts > 1 ? parts : nullptr, n_parts);
     return cudaGetLastError();
@@ -707,6 +753,7 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
+    note_launch();
     permute_kernel<<<1, PERM_THREADS, smem, s>>>(a, WR);
     return cudaGetLastError();
 }
@@ -727,8 +774,11 @@ cudaError_t launch_permute_multi(const PermuteArgs& a, int32_t* hist, cudaStream
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
+    note_launch();
     permute_count_kernel<<<nb, PERM_TB, smem_c, s>>>(a, hist);
+    note_launch();
     permute_scan_kernel<<<1, PERM_THREADS, (PERM_SCAN_CAP + 64) * 4, s>>>(a, hist, nb);
+    note_launch();
     permute_scatter_kernel<<<nb, PERM_TB, 2 * smem_c, s>>>(a, hist);
     return cudaGetLastError();
 }
@@ -737,6 +787,7 @@ cudaError_t launch_gather(const void* x, bool x_f32, int d, const int32_t* row_t
                           int max_rows, __nv_bfloat16* x_perm, int n_sm, cudaStream_t s) {
     int grid = max_rows < n_sm * 8 ? max_rows : n_sm * 8;
     if (grid < 1) grid = 1;
+    note_launch();
     gather_rows_kernel<<<grid, 256, 0, s>>>(x, x_f32 ? 1 : 0, d, row_tok, n_rows_dev, x_perm);
     return cudaGetLastError();
 }
@@ -746,7 +797,14 @@ cudaError_t launch_finalize_bf16(const float* acc, __nv_bfloat16* y, size_t n, b
     size_t grid = (n8 + 255) / 256;
     if (grid > 148 * 16) grid = 148 * 16;
     if (grid < 1) grid = 1;
+    note_launch();
     finalize_kernel<<<(unsigned)grid, 256, 0, s>>>(acc, y, n8, accumulate ? 1 : 0);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_update_bias(const int32_t* counts, int E, float* bias, float gamma, cudaStream_t s) {
+    note_launch();
+    update_bias_kernel<<<1, 1024, 0, s>>>(counts, E, bias, gamma);
     return cudaGetLastError();
 }
 

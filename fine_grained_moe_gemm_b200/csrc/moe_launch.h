@@ -98,6 +98,10 @@ cudaError_t launch_gemm2(int mode, const GemmArgs* args, int grid, cudaStream_t 
 // CTA-pair FP8 grouped GEMM, 128 token rows per item; grid even.
 cudaError_t launch_gemm2_fp8(int mode, const GemmArgs* args, int grid, cudaStream_t s);
 cudaError_t launch_gemm_fp8(int mode, int bn, const GemmArgs* args, int grid, cudaStream_t s);
+// number of kernels launched so far (every launcher counts its launches)
+unsigned long long launch_count();
+// bias[e] -/+= gamma by counts[e] against the mean count
+cudaError_t launch_update_bias(const int32_t* counts, int E, float* bias, float gamma, cudaStream_t s);
 // y[i] = bf16(acc[i] (+ y[i]))
 cudaError_t launch_finalize_bf16(const float* acc, __nv_bfloat16* y, size_t n, bool accumulate, cudaStream_t s);
 cudaError_t read_clear_dev_error(unsigned int* flags, cudaStream_t s);

@@ -173,6 +173,36 @@ MOE_API moe_status moe_forward(const moe_config* cfg, const moe_weights* w, cons
  * for bit.  moe_forward with E4M3 weights runs the same kernel. */
 MOE_API moe_status moe_quantize_act(const void* x, int T, int d, uint8_t* q, float* sx, moe_stream_t stream);
 
+/* Bias controller ("DeepSeek-V3" llm-vis, "MoE router" box, update_bias;
+ * "Teardown: DeepSeek-V3", section 6: after each step the selection bias is
+ * lowered for overloaded experts and raised for underloaded ones).  With the
+ * per-expert token counts of a batch (moe_permute's counts, or the forward's
+ * via moe_routing_out):
+ *   mean = (sum of counts) / E                  (fp32)
+ *   bias[e] = counts[e] > mean ? bias[e] - gamma : bias[e] + gamma   (fp32)
+ * counts: [E] int32; bias: [E] fp32, updated in place; gamma: the step (the
+ * pages use 1e-3).  Deterministic: same inputs, same bits. */
+MOE_API moe_status moe_update_bias(const moe_config* cfg, const int32_t* counts, float* bias, float gamma,
+                                   moe_stream_t stream);
+
+/* The kernels moe_forward runs for T tokens on the current device: which
+ * grouped-GEMM variant, its token tile, the router's K splits, the
+ * permutation's CTA count and how many kernels one call launches.  A pure
+ * host-side query (no launch, no allocation); T == 0 gives all zeros. */
+typedef struct moe_plan {
+    int token_tile;    /* token rows per grouped-GEMM tile (BN: 32, 64, 128 or 256) */
+    int cta_pair;      /* 1: the grouped GEMMs run on CTA pairs (tcgen05 cta_group::2) */
+    int fp8;           /* 1: e4m3 expert GEMMs with block scales */
+    int router_splits; /* K splits of the router GEMM, reduced in a fixed order (1: none) */
+    int permute_ctas;  /* CTAs of the permutation (1: the single-CTA kernel) */
+    int launches;      /* kernels one moe_forward call launches */
+} moe_plan;
+MOE_API moe_status moe_forward_plan(const moe_config* cfg, int T, moe_dtype y_dtype, moe_plan* plan);
+
+/* Number of kernels this library has launched in this process, over all
+ * devices and streams (a diagnostic counter; never reset). */
+MOE_API unsigned long long moe_launch_count(void);
+
 /* Stage timing for moe_forward_ex: six CUDA events (cudaEvent_t handles,
  * created by the caller) that the call records on `stream`:
  *   ev[0] before the router          ev[3] after the gate/up GEMM (SwiGLU)

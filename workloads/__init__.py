@@ -81,9 +81,10 @@ WORKLOADS = {
     "fp8": Workload("fp8", 4, 8192, 7168, 256, 8, 4, 8, 2048, 2048, fp8=True, bias="zero"),
     # Small cases of the same kernels for hardware-counter captures: full width
     # (d = 7168, H = 2048) but 32 experts (2.8 GB of bf16 weights, more than the
-    # L2), with the decode and prefill rows per expert (4 and 128).
+    # L2), with the decode, prefill and FP8 rows per expert (4, 128 and 256).
     "profile_decode": Workload("profile_decode", 5, 16, 7168, 32, 8, 4, 8, 2048, 2048, bias="uniform"),
     "profile_prefill": Workload("profile_prefill", 6, 512, 7168, 32, 8, 4, 8, 2048, 2048, bias="zero"),
+    "profile_fp8": Workload("profile_fp8", 7, 1024, 7168, 32, 8, 4, 8, 2048, 2048, fp8=True, bias="zero"),
 }
 
 # tensor ids of the per-tensor generators
