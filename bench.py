@@ -30,9 +30,17 @@ METRIC = "MoE-layer tokens/sec (T=128 decode, T=4096 prefill); % of HBM/tensor r
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM traffic of the dominant kernel per launch, from one ncu capture, keyed by
-# workload; valid only while the kernel sources hash to the recorded value.
-NCU_TRAFFIC = {}
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
+# kernel per launch, from one ncu capture, keyed by workload; valid only while
+# the kernel sources hash to the recorded value.  profile_decode is captured
+# directly (the gate/up GEMM streams 30 routed + 1 shared expert weight sets);
+# decode is that capture scaled by weight sets streamed, 146 / 31 (traffic grows
+# with the touched experts: the profile_decode capture reads 0.99994 x its
+# algorithmic bytes).
+NCU_TRAFFIC = {
+    "profile_decode": (1_822_874_368, "88be10ddbf705e57"),
+    "decode": (8_585_150_262, "88be10ddbf705e57"),
+}
 
 
 def kernel_source_hash() -> str:
