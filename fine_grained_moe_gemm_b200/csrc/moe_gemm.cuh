@@ -287,6 +287,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) moe_gemm_kernel(const __grid_
             const uint32_t t1 = t0 + BN;
             for (int c0 = 32 * grp; c0 < it.nvalid; c0 += 64) {
                 float v0[32], v1[32];
+                // DOWN: this lane's permuted row (routing coefficient and token), handed
+                // to the other lanes by shuffles: one load a lane instead of one a column
+                float cf_l = 0.0f;
+                int tok_l = 0;
+                if (MODE == GEMM_DOWN && c0 + lane < it.nvalid) {
+                    cf_l = __ldg(&P.row_coef[it.row0 + c0 + lane]);
+                    tok_l = __ldg(&P.row_tok[it.row0 + c0 + lane]);
+                }
                 tmem_ld32x2(t0 + (uint32_t)c0, t1 + (uint32_t)c0, v0, v1);
                 if (MODE == GEMM_GATEUP) {
                     const int f = it.m * 128 + q * 32 + lane;
@@ -300,10 +308,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) moe_gemm_kernel(const __grid_
                     const bool ok0 = f0 < P.ldy, ok1 = f1 < P.ldy;
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
+                        const float cf = __shfl_sync(0xffffffffu, cf_l, jj);
+                        const int tok = __shfl_sync(0xffffffffu, tok_l, jj);
                         if (c0 + jj < it.nvalid) {
-                            const int r = it.row0 + c0 + jj;
-                            const float cf = __ldg(&P.row_coef[r]);
-                            float* yr = P.y + (size_t)__ldg(&P.row_tok[r]) * P.ldy;
+                            float* yr = P.y + (size_t)tok * P.ldy;
                             if (ok0) atomicAdd(yr + f0, v0[jj] * cf);
                             if (ok1) atomicAdd(yr + f1, v1[jj] * cf);
                         }

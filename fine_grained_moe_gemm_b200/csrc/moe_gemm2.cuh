@@ -15,7 +15,7 @@
 // Per item the pair covers GATEUP: 256 features (gate + up accumulators, one
 // CTA per 128 features), DOWN: 512 output features (two 256-row MMAs).
 // Roles per CTA: warp 0 TMA producer, warp 1 TMEM allocator (both CTAs) and
-// MMA issuer (leader CTA only), warps 2-9 epilogue on the CTA's own TMEM.
+// MMA issuer (leader CTA only), warps 2-17 epilogue on the CTA's own TMEM.
 // Synchronisation across the pair: the peer's TMA loads complete on the
 // leader's stage barrier (.cta_group::2 addressing, no multicast); the MMA's
 // commits arrive on the barrier of both CTAs (tcgen05.commit multicast); the
@@ -29,6 +29,13 @@ namespace moe {
 
 constexpr int PAIR_BN = 256;       // token rows per item (whole pair)
 constexpr int PAIR_BOX_ROWS = 16;  // token rows per B TMA box (each CTA loads N/2 rows)
+// Sixteen epilogue warps (four per TMEM lane quarter): the accumulators are
+// single-buffered, so the MMA of the next item waits for the epilogue to drain
+// them, and four warps per SM sub-partition drain them about twice as fast as
+// two.  576 threads leave 112 registers a thread.
+constexpr int PAIR_EPI_WARPS = 16;
+constexpr int PAIR_EPI_THREADS = PAIR_EPI_WARPS * 32;
+constexpr int PAIR_THREADS = 64 + PAIR_EPI_THREADS;
 
 struct Gemm2Cfg {
     static constexpr int A_TILE = 128 * 128;
@@ -121,7 +128,7 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr) {
 }
 
 template <int MODE>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
     moe_gemm2_kernel(const __grid_constant__ GemmArgs P) {
     using C = Gemm2Cfg;
     extern __shared__ uint8_t smem_raw[];
@@ -148,7 +155,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
             mbar_init(&empty[s], 1);
         }
         mbar_init(tfull, 1);
-        mbar_init(tempty, 2 * GEMM_EPI_THREADS / 32);
+        mbar_init(tempty, 2 * PAIR_EPI_WARPS);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -274,13 +281,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         for (int i = cluster_id; i < total; i += n_clusters, ++n_done) {
             const Item it = decode_item<PAIR_BN>(P, i);
             if (et == 0) epi_ok[n_done & 1] = mbar_wait_bounded(tfull, acc_phase, abort_flag) ? 1 : 0;
-            named_bar_sync(1, GEMM_EPI_THREADS);
+            named_bar_sync(1, PAIR_EPI_THREADS);
             if (!epi_ok[n_done & 1]) break;
             tc_fence_after();
             const uint32_t t0 = tmem_base + ((uint32_t)(q * 32) << 16);
             const uint32_t t1 = t0 + PAIR_BN;
-            for (int c0 = 32 * grp; c0 < it.nvalid; c0 += 64) {
+            for (int c0 = 32 * grp; c0 < it.nvalid; c0 += 32 * (PAIR_EPI_WARPS / 4)) {
                 float v0[32], v1[32];
+                // DOWN: this lane's permuted row (routing coefficient and token), handed
+                // to the other lanes by shuffles: one load a lane instead of one a column
+                float cf_l = 0.0f;
+                int tok_l = 0;
+                if (MODE == GEMM_DOWN && c0 + lane < it.nvalid) {
+                    cf_l = __ldg(&P.row_coef[it.row0 + c0 + lane]);
+                    tok_l = __ldg(&P.row_tok[it.row0 + c0 + lane]);
+                }
                 tmem_ld32x2(t0 + (uint32_t)c0, t1 + (uint32_t)c0, v0, v1);
                 if (MODE == GEMM_GATEUP) {
                     const int f = it.m * 256 + (int)rank * 128 + q * 32 + lane;
@@ -294,10 +309,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
                     const bool ok0 = f0 < P.ldy, ok1 = f1 < P.ldy;
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
+                        const float cf = __shfl_sync(0xffffffffu, cf_l, jj);
+                        const int tok = __shfl_sync(0xffffffffu, tok_l, jj);
                         if (c0 + jj < it.nvalid) {
-                            const int r = it.row0 + c0 + jj;
-                            const float cf = __ldg(&P.row_coef[r]);
-                            float* yr = P.y + (size_t)__ldg(&P.row_tok[r]) * P.ldy;
+                            float* yr = P.y + (size_t)tok * P.ldy;
                             if (ok0) atomicAdd(yr + f0, v0[jj] * cf);
                             if (ok1) atomicAdd(yr + f1, v1[jj] * cf);
                         }

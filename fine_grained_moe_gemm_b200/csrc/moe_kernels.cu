@@ -625,11 +625,10 @@ static cudaError_t launch_gemm_fp8_t(const GemmArgs* args, int grid, cudaStream_
 }
 
 int gemm_fp8_smem_bytes(int mode, int bn) {
+    // token tiles of 128 rows and more run on the CTA-pair kernel
     if (mode == MODE_GATEUP)
-        return bn == 32 ? Fp8Cfg<GEMM_GATEUP, 32>::SMEM_BYTES : bn == 64 ? Fp8Cfg<GEMM_GATEUP, 64>::SMEM_BYTES
-                                                                         : Fp8Cfg<GEMM_GATEUP, 128>::SMEM_BYTES;
-    return bn == 32 ? Fp8Cfg<GEMM_DOWN, 32>::SMEM_BYTES : bn == 64 ? Fp8Cfg<GEMM_DOWN, 64>::SMEM_BYTES
-                                                                   : Fp8Cfg<GEMM_DOWN, 128>::SMEM_BYTES;
+        return bn == 32 ? Fp8Cfg<GEMM_GATEUP, 32>::SMEM_BYTES : Fp8Cfg<GEMM_GATEUP, 64>::SMEM_BYTES;
+    return bn == 32 ? Fp8Cfg<GEMM_DOWN, 32>::SMEM_BYTES : Fp8Cfg<GEMM_DOWN, 64>::SMEM_BYTES;
 }
 
 cudaError_t launch_gemm_fp8(int mode, int bn, const GemmArgs* args, int grid, cudaStream_t s) {
@@ -637,13 +636,11 @@ cudaError_t launch_gemm_fp8(int mode, int bn, const GemmArgs* args, int grid, cu
         switch (bn) {
             case 32: return launch_gemm_fp8_t<GEMM_GATEUP, 32>(args, grid, s);
             case 64: return launch_gemm_fp8_t<GEMM_GATEUP, 64>(args, grid, s);
-            case 128: return launch_gemm_fp8_t<GEMM_GATEUP, 128>(args, grid, s);
         }
     } else if (mode == MODE_DOWN) {
         switch (bn) {
             case 32: return launch_gemm_fp8_t<GEMM_DOWN, 32>(args, grid, s);
             case 64: return launch_gemm_fp8_t<GEMM_DOWN, 64>(args, grid, s);
-            case 128: return launch_gemm_fp8_t<GEMM_DOWN, 128>(args, grid, s);
         }
     }
     return cudaErrorInvalidValue;
@@ -661,7 +658,7 @@ static cudaError_t launch_gemm2_t(const GemmArgs* args, int grid, cudaStream_t s
         attr_set[dev] = true;
     }
     note_launch();
-    moe_gemm2_kernel<MODE><<<grid, GEMM_THREADS, Gemm2Cfg::SMEM_BYTES, s>>>(*args);
+    moe_gemm2_kernel<MODE><<<grid, PAIR_THREADS, Gemm2Cfg::SMEM_BYTES, s>>>(*args);
     return cudaGetLastError();
 }
 
