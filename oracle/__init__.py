@@ -74,6 +74,7 @@ def lib():
             L.orc_permute.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P]
             L.orc_quant_act.argtypes = [P, ctypes.c_int, ctypes.c_int, P, P]
             L.orc_update_bias.argtypes = [P, ctypes.c_int, P, ctypes.c_float]
+            L.orc_rmsnorm.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_double, P]
             L.orc_expert_tokens.restype = ctypes.c_int
             L.orc_expert_tokens.argtypes = [ctypes.POINTER(OrcLayer), P, P, P, P, ctypes.c_int, ctypes.c_int, P]
             L.orc_expert_single.argtypes = [ctypes.POINTER(OrcLayer), ctypes.c_int, P, P]
@@ -172,6 +173,21 @@ def update_bias(counts: np.ndarray, bias: np.ndarray, gamma: float = 1e-3) -> np
     b = np.ascontiguousarray(bias, dtype=np.float32).copy()
     lib().orc_update_bias(_ptr(c), c.size, _ptr(b), float(np.float32(gamma)))
     return b
+
+
+RMS_EPS = float(np.float32(1e-6))  # the page's eps, as the fp32 value an fp32 tensor adds
+
+
+def rmsnorm(h_bf16: np.ndarray, g_bf16: np.ndarray, eps: float = RMS_EPS) -> np.ndarray:
+    """Pre-norm ("RMSNorm" box): bf16(bf16(h * r) * g), r = 1/sqrt(mean(h^2) + eps) in fp64.
+    Inputs and output are bf16 bit patterns (uint16)."""
+    h = np.ascontiguousarray(h_bf16, dtype=np.uint16)
+    g = np.ascontiguousarray(g_bf16, dtype=np.uint16)
+    T, d = h.shape
+    assert g.shape == (d,)
+    out = np.empty((T, d), dtype=np.uint16)
+    lib().orc_rmsnorm(_ptr(h), _ptr(g), T, d, float(eps), _ptr(out))
+    return out
 
 
 def quant_act(x_bf16: np.ndarray):

@@ -313,6 +313,32 @@ void orc_update_bias(const int32_t* counts, int E, float* bias, float gamma)
 }
 
 /* ------------------------------------------------------------------------ */
+/* Pre-norm of the MoE sublayer ("DeepSeek-V3" llm-vis, "RMSNorm" box: each  */
+/* token vector is rescaled to unit RMS over its features, eps 1e-6, the     */
+/* normalised value is cast back to the activation dtype, then multiplied by */
+/* the learned per-feature gain; "Residual add" box: y = h + ffn(norm2(h))): */
+/*   r      = 1 / sqrt(mean_c h[c]^2 + eps)      (fp64 here; fp32 on the page)*/
+/*   out[c] = bf16( bf16(h[c] * r) * g[c] )                                   */
+/* ------------------------------------------------------------------------ */
+
+void orc_rmsnorm(const uint16_t* h, const uint16_t* g, int T, int d, double eps, uint16_t* out)
+{
+    for (int t = 0; t < T; ++t) {
+        const uint16_t* hr = h + (int64_t)t * d;
+        double ss = 0.0;
+        for (int c = 0; c < d; ++c) {
+            double v = orc_bf16_to_f64(hr[c]);
+            ss += v * v;
+        }
+        double r = 1.0 / sqrt(ss / (double)d + eps);
+        for (int c = 0; c < d; ++c) {
+            uint16_t v = orc_bf16_from_f64(orc_bf16_to_f64(hr[c]) * r);
+            out[(int64_t)t * d + c] = orc_bf16_from_f64(orc_bf16_to_f64(v) * orc_bf16_to_f64(g[c]));
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* S6  activation quantisation (teardown, section 10: activations scaled in  */
 /* 1x128 tiles, E4M3).  Per token and 128-channel block, in fp32:            */
 /*   sx = amax / 448 (1 when amax = 0);  q = e4m3_rn_sat(x / sx).            */
