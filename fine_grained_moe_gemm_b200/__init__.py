@@ -77,6 +77,13 @@ def lib():
             L.moe_forward_ex.restype = I
             L.moe_forward_ex.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, I, P, I, I, P,
                                          ctypes.c_size_t, P, P, P]
+            L.moe_rmsnorm.restype = I
+            L.moe_rmsnorm.argtypes = [P, P, ctypes.c_float, I, I, P, P, P, P]
+            L.moe_block_workspace_size.restype = ctypes.c_size_t
+            L.moe_block_workspace_size.argtypes = [ctypes.POINTER(MoeConfig), I]
+            L.moe_forward_block.restype = I
+            L.moe_forward_block.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, ctypes.c_float,
+                                            P, P, I, P, P, ctypes.c_size_t, P, P, P]
             L.moe_forward_plan.restype = I
             L.moe_forward_plan.argtypes = [ctypes.POINTER(MoeConfig), I, I, ctypes.c_void_p]
             L.moe_launch_count.restype = ctypes.c_ulonglong
@@ -193,6 +200,29 @@ def forward_plan(cfg: MoeConfig, T: int, y_dtype=torch.bfloat16) -> dict:
     return {n: getattr(plan, n) for n, _ in MoePlan._fields_}
 
 
+def _events(stage_events):
+    if stage_events is None:
+        return None
+    ev = MoeStageEvents()
+    for i, e in enumerate(stage_events):
+        if e is not None and e.cuda_event == 0:
+            e.record()  # torch creates the underlying event lazily
+        ev.ev[i] = e.cuda_event if e is not None else None
+    return ev
+
+
+def _routing(routing_out):
+    if routing_out is None:
+        return None
+    ro = MoeRoutingOut()
+    for name, _ in MoeRoutingOut._fields_:
+        t = routing_out.get(name)
+        if t is not None:
+            _dev(t, name)
+            setattr(ro, name, t.data_ptr())
+    return ro
+
+
 def moe_forward(cfg: MoeConfig, weights, x, bias, y, accumulate: bool = False, workspace=None, stream=None,
                 stage_events=None, routing_out=None):
     """y (+)= MoE(x).  ``weights`` is a MoeWeights or a dict of tensors; ``workspace`` a uint8 CUDA tensor of at
@@ -205,21 +235,7 @@ def moe_forward(cfg: MoeConfig, weights, x, bias, y, accumulate: bool = False, w
     mw = weights if isinstance(weights, MoeWeights) else make_weights(weights)
     T = x.shape[0]
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    ev = None
-    if stage_events is not None:
-        ev = MoeStageEvents()
-        for i, e in enumerate(stage_events):
-            if e is not None and e.cuda_event == 0:
-                e.record()  # torch creates the underlying event lazily
-            ev.ev[i] = e.cuda_event if e is not None else None
-    ro = None
-    if routing_out is not None:
-        ro = MoeRoutingOut()
-        for name, _ in MoeRoutingOut._fields_:
-            t = routing_out.get(name)
-            if t is not None:
-                _dev(t, name)
-                setattr(ro, name, t.data_ptr())
+    ev, ro = _events(stage_events), _routing(routing_out)
     _check(lib().moe_forward_ex(ctypes.byref(cfg), ctypes.byref(mw), _p(x), _p(bias), T, _p(y), _dtype_code(y),
                                 1 if accumulate else 0, _p(workspace), ws_bytes, _stream(stream),
                                 ctypes.byref(ev) if ev is not None else None,
@@ -237,6 +253,39 @@ def moe_update_bias(cfg: MoeConfig, counts, bias, gamma: float = 1e-3, stream=No
         _dev(t, n)
     _check(lib().moe_update_bias(ctypes.byref(cfg), _p(counts), _p(bias), float(gamma), _stream(stream)),
            "moe_update_bias")
+
+
+RMS_EPS = 1e-6
+
+
+def block_workspace_size(cfg: MoeConfig, T: int) -> int:
+    return int(lib().moe_block_workspace_size(ctypes.byref(cfg), int(T)))
+
+
+def moe_rmsnorm(h, g, out, q=None, sx=None, eps: float = RMS_EPS, stream=None):
+    """out = bf16(bf16(h * r) * g), r = 1/sqrt(mean(h^2) + eps) per row of bf16 h [T, d]; with q (uint8 [T, d])
+    and sx (fp32 [T, d/128]) also the e4m3 activation codes and scales of out."""
+    for n, t in (("h", h), ("g", g), ("out", out), ("q", q), ("sx", sx)):
+        _dev(t, n)
+    T, d = h.shape
+    _check(lib().moe_rmsnorm(_p(h), _p(g), float(eps), T, d, _p(out), _p(q), _p(sx), _stream(stream)),
+           "moe_rmsnorm")
+
+
+def moe_forward_block(cfg: MoeConfig, weights, norm_g, h, bias, y, eps: float = RMS_EPS, workspace=None,
+                      stream=None, stage_events=None, routing_out=None):
+    """y = bf16(h + MoE(RMSNorm(h))) for the bf16 residual stream h [T, d]; y may be h itself.  ``workspace``: at
+    least ``block_workspace_size(cfg, T)`` bytes.  ``stage_events`` / ``routing_out`` as in ``moe_forward``."""
+    for n, t in (("norm_g", norm_g), ("h", h), ("bias", bias), ("y", y), ("workspace", workspace)):
+        _dev(t, n)
+    mw = weights if isinstance(weights, MoeWeights) else make_weights(weights)
+    T = h.shape[0]
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    ev, ro = _events(stage_events), _routing(routing_out)
+    _check(lib().moe_forward_block(ctypes.byref(cfg), ctypes.byref(mw), _p(norm_g), float(eps), _p(h), _p(bias), T,
+                                   _p(y), _p(workspace), ws_bytes, _stream(stream),
+                                   ctypes.byref(ev) if ev is not None else None,
+                                   ctypes.byref(ro) if ro is not None else None), "moe_forward_block")
 
 
 def moe_quantize_act(x, q, sx, stream=None):

@@ -288,6 +288,13 @@ moe_status route_impl(const moe_config* c, const DevInfo& di, const void* x, con
                                      part, n_parts));
 }
 
+size_t xhat_bytes(const moe_config* c, int T) { return ((size_t)T * c->d * 2 + 255) & ~(size_t)255; }
+
+moe_status forward_impl(const moe_config* cfg, const moe_weights* wt, const void* x, const float* bias, int T,
+                        void* y, moe_dtype y_dtype, int accumulate, void* workspace, size_t ws_bytes,
+                        moe_stream_t stream, const moe_stage_events* events, const moe_routing_out* routing,
+                        const void* norm_g, float eps);
+
 }  // namespace
 
 extern "C" {
@@ -398,6 +405,50 @@ moe_status moe_forward(const moe_config* cfg, const moe_weights* wt, const void*
 moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const void* x, const float* bias, int T,
                           void* y, moe_dtype y_dtype, int accumulate, void* workspace, size_t ws_bytes,
                           moe_stream_t stream, const moe_stage_events* events, const moe_routing_out* routing) {
+    return forward_impl(cfg, wt, x, bias, T, y, y_dtype, accumulate, workspace, ws_bytes, stream, events, routing,
+                        nullptr, 0.0f);
+}
+
+size_t moe_block_workspace_size(const moe_config* cfg, int T_max) {
+    const size_t base = moe_workspace_size(cfg, T_max);
+    return base ? base + xhat_bytes(cfg, T_max) : 0;
+}
+
+moe_status moe_rmsnorm(const void* h, const void* g, float eps, int T, int d, void* out, uint8_t* q, float* sx,
+                       moe_stream_t stream) {
+    if (T < 0 || d <= 0 || d % 8 || d > 8 * NORM_MAX_VEC * NORM_THREADS || !(eps >= 0.0f)) return MOE_ERR_INVALID_ARG;
+    if ((q != nullptr) != (sx != nullptr) || (q && d % 128)) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!h || !g || !out || !aligned16(h) || !aligned16(g) || !aligned16(out) || (q && (!aligned16(q) || !aligned16(sx))))
+        return MOE_ERR_INVALID_ARG;
+    DevInfo di;
+    moe_status st = check_device(&di);
+    if (st != MOE_OK) return st;
+    return cuda_status(launch_rmsnorm(static_cast<const __nv_bfloat16*>(h), static_cast<const __nv_bfloat16*>(g), T,
+                                      d, eps, static_cast<__nv_bfloat16*>(out), q, sx, (cudaStream_t)stream));
+}
+
+moe_status moe_forward_block(const moe_config* cfg, const moe_weights* wt, const void* norm_g, float eps,
+                             const void* h, const float* bias, int T, void* y, void* workspace, size_t ws_bytes,
+                             moe_stream_t stream, const moe_stage_events* events, const moe_routing_out* routing) {
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (cfg->act_dtype != MOE_BF16 || cfg->d > 8 * NORM_MAX_VEC * NORM_THREADS) return MOE_ERR_UNSUPPORTED;
+    if (T < 0 || !(eps >= 0.0f)) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!norm_g || !aligned16(norm_g)) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < moe_block_workspace_size(cfg, T)) return MOE_ERR_WORKSPACE;
+    return forward_impl(cfg, wt, h, bias, T, y, MOE_BF16, 0, workspace, ws_bytes, stream, events, routing, norm_g, eps);
+}
+
+}  // extern "C"
+
+namespace {
+
+moe_status forward_impl(const moe_config* cfg, const moe_weights* wt, const void* x, const float* bias, int T,
+                        void* y, moe_dtype y_dtype, int accumulate, void* workspace, size_t ws_bytes,
+                        moe_stream_t stream, const moe_stage_events* events, const moe_routing_out* routing,
+                        const void* norm_g, float eps) {
     moe_status st = check_config(cfg);
     if (st != MOE_OK) return st;
     if (T < 0 || (y_dtype != MOE_F32 && y_dtype != MOE_BF16) || (accumulate != 0 && accumulate != 1))
@@ -455,8 +506,19 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     auto mark = [&](int i) {
         if (events && events->ev[i]) cudaEventRecord((cudaEvent_t)events->ev[i], s);
     };
-    // (1)+(2) router and selection
+    // (0) pre-norm of the sublayer: the layer runs on x = RMSNorm(h) and adds h back at
+    //     the end; in the FP8 layer the same pass writes the activation codes and scales
     mark(0);
+    const void* residual = accumulate ? y : nullptr;
+    if (norm_g) {
+        __nv_bfloat16* xhat = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(workspace) + W.bytes);
+        if (launch_rmsnorm(static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(norm_g), T, d,
+                           eps, xhat, fp8 ? W.x_q : nullptr, fp8 ? W.sx : nullptr, s) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        residual = x;
+        x = xhat;
+    }
+    // (1)+(2) router and selection
     st = route_impl(cfg, di, x, wt->w_router, W.logits, bias, T, W.idx, W.w, s, W.part, plan.router_parts);
     if (st != MOE_OK) return st;
     mark(1);
@@ -487,7 +549,7 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     const cudaError_t ep = plan.permute_multi ? launch_permute_multi(pa, W.hist, s) : launch_permute(pa, s);
     if (ep != cudaSuccess) return MOE_ERR_CUDA;
     if (fp8) {
-        if (launch_quant_act(static_cast<const __nv_bfloat16*>(x), T, d, W.x_q, W.sx, s) != cudaSuccess ||
+        if ((!norm_g && launch_quant_act(static_cast<const __nv_bfloat16*>(x), T, d, W.x_q, W.sx, s) != cudaSuccess) ||
             launch_gather_fp8(W.x_q, W.sx, d, W.row_tok, W.row_off + NG, rows_max, W.xq_perm, W.sxT, di.sm_count,
                               s) != cudaSuccess)
             return MOE_ERR_CUDA;
@@ -589,12 +651,16 @@ moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const vo
     mark(4);
 
     if (y_dtype == MOE_BF16 &&
-        launch_finalize_bf16(W.y_acc, static_cast<__nv_bfloat16*>(y), (size_t)T * d, accumulate != 0, s) !=
-            cudaSuccess)
+        launch_finalize_bf16(W.y_acc, static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(y),
+                             (size_t)T * d, s) != cudaSuccess)
         return MOE_ERR_CUDA;
     mark(5);
     return MOE_OK;
 }
+
+}  // namespace
+
+extern "C" {
 
 moe_status moe_device_error(unsigned int* flags, moe_stream_t stream) {
     if (!flags) return MOE_ERR_INVALID_ARG;

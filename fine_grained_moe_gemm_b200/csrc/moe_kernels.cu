@@ -13,6 +13,7 @@
 //   moe_gemm2_kernel      CTA-pair grouped GEMM, cta_group::2 (moe_gemm2.cuh)
 //   moe_gemm2_fp8_kernel  CTA-pair e4m3 GEMM (moe_gemm2_fp8.cuh)
 //   update_bias_kernel    selection-bias controller step
+//   rmsnorm_kernel        pre-norm of the sublayer (+ the 1x128 e4m3 quantisation)
 //   finalize_kernel       fp32 combine buffer -> bf16 output (+ residual)
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -501,6 +502,87 @@ __global__ void __launch_bounds__(256) gather_fp8_kernel(const uint8_t* __restri
     }
 }
 
+// ============================================================================ pre-norm
+// "RMSNorm" box: r = 1/sqrt(mean_c h[c]^2 + eps), the mean reduced in fp32;
+// out = bf16(bf16(h * r) * g).  With q and sx the same pass also writes the
+// 1x128 e4m3 codes and scales of out, in the arithmetic of quant_act_kernel.
+// One CTA of 128 threads per token row; vector i of 8 features goes to thread
+// i % 128, so a 128-feature block is 16 consecutive lanes of one warp.
+__global__ void __launch_bounds__(NORM_THREADS) rmsnorm_kernel(const __nv_bfloat16* __restrict__ h,
+                                                               const __nv_bfloat16* __restrict__ g, int d, float eps,
+                                                               __nv_bfloat16* __restrict__ out,
+                                                               uint8_t* __restrict__ q, float* __restrict__ sx) {
+    __shared__ float s_part[NORM_THREADS / 32];
+    const int t = blockIdx.x;
+    const int lane = threadIdx.x & 31;
+    const int nvec = d / 8;
+    const uint4* hr = reinterpret_cast<const uint4*>(h + (size_t)t * d);
+    uint4 v[NORM_MAX_VEC];
+    float ss = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NORM_MAX_VEC; ++i) {
+        const int vi = threadIdx.x + i * NORM_THREADS;
+        v[i] = vi < nvec ? hr[vi] : make_uint4(0u, 0u, 0u, 0u);
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v[i]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(p2[j]);
+            ss = fmaf(f.x, f.x, ss);
+            ss = fmaf(f.y, f.y, ss);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) s_part[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    float tot = 0.0f;
+#pragma unroll
+    for (int w = 0; w < NORM_THREADS / 32; ++w) tot += s_part[w];
+    const float r = __frsqrt_rn(__fadd_rn(__fdiv_rn(tot, (float)d), eps));
+    const uint4* gv = reinterpret_cast<const uint4*>(g);
+    uint4* ov = reinterpret_cast<uint4*>(out + (size_t)t * d);
+#pragma unroll
+    for (int i = 0; i < NORM_MAX_VEC; ++i) {
+        const int vi = threadIdx.x + i * NORM_THREADS;
+        if (i * NORM_THREADS >= nvec) break;  // uniform over the CTA
+        const bool ok = vi < nvec;
+        const uint4 gg = ok ? gv[vi] : make_uint4(0u, 0u, 0u, 0u);
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v[i]);
+        const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gg);
+        float o[8];
+        uint32_t pk[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(p2[j]);
+            const float2 gf = __bfloat1622float2(g2[j]);
+            const float a0 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(f.x, r)));
+            const float a1 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(f.y, r)));
+            const __nv_bfloat162 b = __floats2bfloat162_rn(__fmul_rn(a0, gf.x), __fmul_rn(a1, gf.y));
+            const float2 bf = __bfloat1622float2(b);
+            o[2 * j] = bf.x;
+            o[2 * j + 1] = bf.y;
+            pk[j] = *reinterpret_cast<const uint32_t*>(&b);
+        }
+        if (ok) ov[vi] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        if (q) {
+            float amax = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(o[j]));
+#pragma unroll
+            for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+            const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+            uint32_t c[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) c[j] = cvt_e4m3x2(__fdiv_rn(o[2 * j + 1], scale), __fdiv_rn(o[2 * j], scale));
+            if (ok) {
+                *reinterpret_cast<uint2*>(q + (size_t)t * d + (size_t)vi * 8) =
+                    make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+                if ((vi & 15) == 0) sx[(size_t)t * (d / 128) + vi / 16] = scale;
+            }
+        }
+    }
+}
+
 // ============================================================================ bias controller
 // "MoE router" box, update_bias: mean = sum(counts) / E in fp32; experts above
 // it get bias - gamma, the others bias + gamma (one correctly rounded fp32 op).
@@ -526,15 +608,17 @@ __global__ void __launch_bounds__(1024) update_bias_kernel(const int32_t* __rest
 }
 
 // ============================================================================ finalize
-__global__ void __launch_bounds__(256) finalize_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ y,
-                                                       size_t n8, int accumulate) {
+// y = bf16(acc (+ residual)); residual may be y itself (an in-place update of the
+// residual stream: each element is read before it is written, by the same thread).
+__global__ void __launch_bounds__(256) finalize_kernel(const float* __restrict__ acc, const __nv_bfloat16* residual,
+                                                       __nv_bfloat16* y, size_t n8) {
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {
         float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
         float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
         float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
         uint4* yp = reinterpret_cast<uint4*>(y) + i;
-        if (accumulate) {
-            uint4 old = *yp;
+        if (residual) {
+            uint4 old = reinterpret_cast<const uint4*>(residual)[i];
             const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&old);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -789,13 +873,21 @@ cudaError_t launch_gather(const void* x, bool x_f32, int d, const int32_t* row_t
     return cudaGetLastError();
 }
 
-cudaError_t launch_finalize_bf16(const float* acc, __nv_bfloat16* y, size_t n, bool accumulate, cudaStream_t s) {
+cudaError_t launch_finalize_bf16(const float* acc, const __nv_bfloat16* residual, __nv_bfloat16* y, size_t n,
+                                 cudaStream_t s) {
     size_t n8 = n / 8;
     size_t grid = (n8 + 255) / 256;
     if (grid > 148 * 16) grid = 148 * 16;
     if (grid < 1) grid = 1;
     note_launch();
-    finalize_kernel<<<(unsigned)grid, 256, 0, s>>>(acc, y, n8, accumulate ? 1 : 0);
+    finalize_kernel<<<(unsigned)grid, 256, 0, s>>>(acc, residual, y, n8);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rmsnorm(const __nv_bfloat16* h, const __nv_bfloat16* g, int T, int d, float eps,
+                           __nv_bfloat16* out, uint8_t* q, float* sx, cudaStream_t s) {
+    note_launch();
+    rmsnorm_kernel<<<T, NORM_THREADS, 0, s>>>(h, g, d, eps, out, q, sx);
     return cudaGetLastError();
 }
 

@@ -103,7 +103,13 @@ unsigned long long launch_count();
 // bias[e] -/+= gamma by counts[e] against the mean count
 cudaError_t launch_update_bias(const int32_t* counts, int E, float* bias, float gamma, cudaStream_t s);
 // y[i] = bf16(acc[i] (+ y[i]))
-cudaError_t launch_finalize_bf16(const float* acc, __nv_bfloat16* y, size_t n, bool accumulate, cudaStream_t s);
+cudaError_t launch_finalize_bf16(const float* acc, const __nv_bfloat16* residual, __nv_bfloat16* y, size_t n,
+                                 cudaStream_t s);
+// pre-norm: out = bf16(bf16(h * r) * g) per token row (+ e4m3 codes / scales when q, sx are set)
+constexpr int NORM_THREADS = 128;
+constexpr int NORM_MAX_VEC = 8;  // 8-feature vectors per thread: d <= 8 * 8 * 128
+cudaError_t launch_rmsnorm(const __nv_bfloat16* h, const __nv_bfloat16* g, int T, int d, float eps,
+                           __nv_bfloat16* out, uint8_t* q, float* sx, cudaStream_t s);
 cudaError_t read_clear_dev_error(unsigned int* flags, cudaStream_t s);
 
 }  // namespace moe

@@ -238,6 +238,35 @@ MOE_API moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* w, c
                                   size_t ws_bytes, moe_stream_t stream, const moe_stage_events* events,
                                   const moe_routing_out* routing);
 
+/* Pre-norm ("DeepSeek-V3" llm-vis, "RMSNorm" box: every token vector is
+ * rescaled to unit RMS over its features with eps = 1e-6, cast back to bf16,
+ * then multiplied by the learned per-feature gain):
+ *   r_t      = 1 / sqrt(mean_c h[t,c]^2 + eps)      (fp32 reduction, correctly
+ *                                                    rounded divide and rsqrt)
+ *   out[t,c] = bf16( bf16(h[t,c] * r_t) * g[c] )
+ * h, out: [T, d] bf16 row-major (must not overlap); g: [d] bf16; all 16-byte
+ * aligned; d a multiple of 8 and at most 8192.  With q and sx (both or
+ * neither; d a multiple of 128) the same pass also writes the 1x128 e4m3 codes
+ * and scales of `out`, bit for bit as moe_quantize_act(out) would. */
+MOE_API moe_status moe_rmsnorm(const void* h, const void* g, float eps, int T, int d, void* out, uint8_t* q,
+                               float* sx, moe_stream_t stream);
+
+/* The MoE sublayer of a pre-norm decoder block ("Residual add" box: the
+ * sublayer reads norm2(h) and its output is added to the untouched stream h):
+ *   y = bf16( h + MoE(RMSNorm(h; norm_g, eps)) )
+ * with MoE as moe_forward computes it (routing, experts, combine) on the
+ * normalised activations; in the FP8 layer the norm also produces the e4m3
+ * activations (one pass).  h: [T, d] bf16 (cfg->act_dtype must be MOE_BF16);
+ * norm_g: [d] bf16; y: [T, d] bf16 and may be h itself (the residual stream
+ * updated in place).  workspace: moe_block_workspace_size(cfg, T) bytes,
+ * 256-byte aligned.  events / routing as in moe_forward_ex (the norm runs in
+ * the first stage). */
+MOE_API size_t moe_block_workspace_size(const moe_config* cfg, int T_max);
+MOE_API moe_status moe_forward_block(const moe_config* cfg, const moe_weights* w, const void* norm_g, float eps,
+                                     const void* h, const float* bias, int T, void* y, void* workspace,
+                                     size_t ws_bytes, moe_stream_t stream, const moe_stage_events* events,
+                                     const moe_routing_out* routing);
+
 /* Size of the device scratch array that moe_forward_noalloc uses in place of
  * a caller-provided workspace: 32 MiB.  At the DeepSeek-V3 sizes (d = 7168,
  * 256 experts, top-8, H = Hs = 2048, one shared expert) that holds up to

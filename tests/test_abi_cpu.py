@@ -101,3 +101,28 @@ def test_no_device_means_unsupported_not_fallback(L):
     P = ctypes.c_void_p
     st = L.moe_permute(ctypes.byref(cfg), P(16), 4, P(16), P(16), P(16), P(16), None)
     assert st == moe.MOE_ERR_UNSUPPORTED
+
+
+def test_prenorm_and_block_arguments(L):
+    cfg = cfg_of(WORKLOADS["decode"])
+    P = ctypes.c_void_p
+    F = ctypes.c_float
+    # moe_rmsnorm: negative T, d not a multiple of 8, q without sx, fp8 outputs with d % 128, misaligned h
+    assert L.moe_rmsnorm(P(16), P(16), F(1e-6), -1, 7168, P(16), None, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_rmsnorm(P(16), P(16), F(1e-6), 4, 7164, P(16), None, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_rmsnorm(P(16), P(16), F(1e-6), 4, 7168, P(16), P(16), None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_rmsnorm(P(16), P(16), F(1e-6), 4, 200, P(16), P(16), P(16), None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_rmsnorm(P(18), P(16), F(1e-6), 4, 7168, P(16), None, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_rmsnorm(P(16), P(16), F(-1.0), 4, 7168, P(16), None, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_rmsnorm(None, None, F(1e-6), 0, 7168, None, None, None, None) == moe.MOE_OK
+    # the block workspace holds the forward's plus the normalised activations
+    for T in (1, 128, 4096):
+        assert L.moe_block_workspace_size(ctypes.byref(cfg), T) >= moe.workspace_size(cfg, T) + T * 7168 * 2
+    w = moe.MoeWeights(w_router=16, w_gate=16, w_up=16, w_down=16, ws_gate=16, ws_up=16, ws_down=16)
+    blk = lambda c, g, ws: L.moe_forward_block(ctypes.byref(c), ctypes.byref(w), g, F(1e-6), P(16), P(16), 4, P(16),
+                                              P(1024), ws, None, None, None)
+    assert blk(cfg, P(16), 1024) == moe.MOE_ERR_WORKSPACE
+    assert blk(cfg, None, 1 << 30) == moe.MOE_ERR_INVALID_ARG          # no gain
+    assert blk(cfg, P(20), 1 << 30) == moe.MOE_ERR_INVALID_ARG         # misaligned gain
+    f32 = cfg_of(WORKLOADS["tiny"])                                     # fp32 activations: not a bf16 stream
+    assert blk(f32, P(16), 1 << 30) == moe.MOE_ERR_UNSUPPORTED

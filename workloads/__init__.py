@@ -89,7 +89,7 @@ WORKLOADS = {
 
 # tensor ids of the per-tensor generators
 _TID = {"x": 1, "w_router": 2, "bias": 3, "w_gate": 4, "w_up": 5, "w_down": 6,
-        "ws_gate": 7, "ws_up": 8, "ws_down": 9, "hot": 10, "residual": 11}
+        "ws_gate": 7, "ws_up": 8, "ws_down": 9, "hot": 10, "residual": 11, "norm_g": 12}
 
 WEIGHT_STD = 0.02
 BIAS_RANGE = 0.1
@@ -158,6 +158,19 @@ def make_residual(wl: Workload, device="cpu", seed: int = 0, T: int | None = Non
     T = wl.T if T is None else T
     g = _gen(device, _seed(seed, wl.wid, "residual", T))
     return torch.randn((T, wl.d), generator=g, device=device, dtype=torch.float32).to(dtype)
+
+
+def make_norm_gain(wl: Workload, device="cpu", seed: int = 0) -> torch.Tensor:
+    """Per-feature gain of the pre-norm, bf16 U[0.5, 1.5] (a trained gain; the pages
+    initialise it to ones)."""
+    g = _gen(device, _seed(seed, wl.wid, "norm_g"))
+    return (torch.rand(wl.d, generator=g, device=device, dtype=torch.float32) + 0.5).to(torch.bfloat16)
+
+
+def make_stream(wl: Workload, device="cpu", seed: int = 0, T: int | None = None, scale: float = 4.0) -> torch.Tensor:
+    """Residual stream h entering the MoE sublayer: bf16 N(0, scale^2) (larger than the
+    normalised activations, as the stream grows with depth)."""
+    return (make_residual(wl, device, seed, T, dtype=torch.float32) * scale).to(torch.bfloat16)
 
 
 def _quantise_blocks_e4m3(w: torch.Tensor):
