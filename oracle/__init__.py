@@ -271,6 +271,23 @@ def expert_tokens(layer: Layer, x: np.ndarray, idx: np.ndarray, w: np.ndarray, t
     return y
 
 
+def dense_ffn(x: np.ndarray, w_gate, w_up, w_down, s_gate=None, s_up=None, s_down=None, tokens=None,
+              x_is_f32=False, n_threads=None) -> np.ndarray:
+    """Dense SwiGLU FFN ("SwiGLU MLP" box; the first layers of the model have a dense FFN
+    of hidden 18432 instead of experts): fp64 y = W_down(SiLU(W_gate x) * (W_up x)) for the
+    listed tokens, h stored in bf16 (e4m3 with 1x128 scales when the weights are e4m3 with
+    128x128 block scales, and x quantised per 1x128 tile).  It is the layer's expert math
+    with no routed expert and the dense weights in the always-on slot."""
+    d = x.shape[1]
+    Hd = np.asarray(w_gate).shape[0]
+    fp8 = s_gate is not None
+    kw = dict(s_gate=[], s_up=[], s_down=[], ss_gate=s_gate, ss_up=s_up, ss_down=s_down) if fp8 else {}
+    L = Layer(d, 0, Hd, Hd, 0, 1.0, [], [], [], w_gate, w_up, w_down, x_is_f32=x_is_f32, **kw)
+    T = x.shape[0]
+    tokens = np.arange(T, dtype=np.int32) if tokens is None else tokens
+    return expert_tokens(L, x, np.zeros((T, 0), np.int32), np.zeros((T, 0), np.float32), tokens, n_threads)
+
+
 def expert_single(layer: Layer, e: int, xh: np.ndarray) -> np.ndarray:
     """One expert (e < 0: shared) on an fp64 input row, for closed-form pins."""
     xh = np.ascontiguousarray(xh, dtype=np.float64)
