@@ -507,6 +507,115 @@ def run_ours(args, wl):
     return 0
 
 
+def run_dense(args, wl):
+    """The dense SwiGLU FFN of the model's first layers (d -> 18432 -> d) on the same
+    grouped-GEMM kernels, at the workload's T (e4m3 weights for the FP8 workload)."""
+    import torch
+    import torch.distributed as dist
+
+    import fine_grained_moe_gemm_b200 as moe
+    from workloads import DENSE_HIDDEN, make_dense_weights, make_x
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    peaks, peak_kind = load_peaks()
+    T, d, Hd = wl.T, wl.d, DENSE_HIDDEN
+    W = make_dense_weights(d, Hd, wl.fp8, dev, seed=rank)
+    x = make_x(wl, dev, seed=rank)
+    act = moe.MOE_BF16
+    wdt = moe.MOE_E4M3 if wl.fp8 else moe.MOE_BF16
+    ws = torch.empty(moe.dense_workspace_size(d, Hd, act, wdt, T), dtype=torch.uint8, device=dev)
+    y = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def forward(xin, ev=None):
+        moe.moe_dense_ffn(W["w_gate"], W["w_up"], W["w_down"], xin, y, W.get("s_gate"), W.get("s_up"),
+                          W.get("s_down"), workspace=ws, stage_events=ev)
+
+    for _ in range(max(args.warmup, 0)):
+        forward(x)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n0 = moe.launch_count()
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for i in range(args.steps):
+            forward(x, evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    launches = moe.launch_count() - n0
+    per_step = 4 + (2 if wl.fp8 else 1)  # tables, gather (+ quantisation), two GEMMs, cast
+    if launches != per_step * args.steps or moe.device_error() != 0:
+        raise RuntimeError(f"dense FFN: {launches} launches, device error word set or not as planned")
+    tt = torch.tensor([t0.elapsed_time(t1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    ms = float(tt.item())
+    stage_ms = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, name in enumerate(moe.STAGES)}
+    # end to end with host buffers
+    x_host, y_host = x.cpu().pin_memory(), torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        e_evs[i][0].record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        forward(x_dev)
+        y_host.copy_(y, non_blocking=True)
+        e_evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    te = torch.tensor([sum(a.elapsed_time(b) for a, b in e_evs)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    wb = 1 if wl.fp8 else 2
+    sc = 3 * (d // 128) * (Hd // 128) * 4 if wl.fp8 else 0
+    F = 2 * 3 * d * Hd * T
+    B = 3 * d * Hd * wb + sc + 2 * T * d * 2
+    sus = ms / 1e3 >= SUSTAINED_AFTER_S
+    step_s = ms / args.steps / 1e3
+    lr = roofline(F, B, step_s, peaks, peak_kind, fp8=wl.fp8, sustained=sus)
+    t_roof = max(F / (tensor_peak(peaks, wl.fp8, sus) * 1e12), B / (peaks["hbm_gbs"] * 1e9))
+    lr.update({"roofline_ms": round(t_roof * 1e3, 4), "frac_of_roofline_time": round(t_roof / step_s, 4),
+               "algorithmic_bytes": B, "algorithmic_flops": F})
+    k_name = max(("gate_up", "down+combine"), key=lambda n: stage_ms[n])
+    if k_name == "gate_up":
+        kF, kB = 2 * 2 * d * Hd * T, 2 * d * Hd * wb + 2 * sc // 3 + T * d * 2 + T * Hd * 2
+    else:
+        kF, kB = 2 * d * Hd * T, d * Hd * wb + sc // 3 + T * Hd * 2 + T * d * 4
+    kr = roofline(kF, kB, stage_ms[k_name] / 1e3, peaks, peak_kind, fp8=wl.fp8, sustained=sus)
+    kr.update({"kernel": k_name + " grouped GEMM (one group of T rows)", "traffic": None,
+               "algorithmic_bytes": kB, "algorithmic_flops": kF})
+    line = {
+        "metric": METRIC, "value": round(world * T * args.steps / (ms / 1e3), 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if wl.fp8 else "bf16",
+        "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights; no checkpoint)",
+        "config": {"workload": f"dense SwiGLU FFN d={d} -> {Hd} -> {d} (the model's first layers), T={T}"
+                               + (", e4m3 weights with 128x128 fp32 block scales" if wl.fp8 else ""),
+                   "T": T, "l2": f"inputs larger than L2: {3 * d * Hd * wb / 1e9:.2f} GB of weights stream every step",
+                   "parallelism": f"replicas x{world} (no data-path collective)"},
+        "roofline": kr, "layer_roofline": lr, "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+        "e2e": {"value": round(world * T * args.steps / (float(te.item()) / 1e3), 1), "unit": UNIT,
+                "h2d_bytes_per_step": x.numel() * x.element_size(), "d2h_bytes_per_step": y.numel() * y.element_size()},
+        "gpu_launches": launches, "clocks": clk.summary(), "kernel_source": kernel_source_hash(),
+    }
+    print(json.dumps(line))
+    return 0
+
+
 def main():
     from workloads import WORKLOADS
 
@@ -519,16 +628,19 @@ def main():
     p.add_argument("--cpu-sample", type=int, default=0, help="tokens of the oracle sample (0: min(T, 8))")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--tokens", type=int, default=0, help="override the workload's T (sweeps; default: as named)")
-    p.add_argument("--op", choices=("layer", "block"), default="layer",
-                   help="layer: y = MoE(x) (moe_forward); block: y = h + MoE(RMSNorm(h)) (moe_forward_block)")
+    p.add_argument("--op", choices=("layer", "block", "dense"), default="layer",
+                   help="layer: y = MoE(x) (moe_forward); block: y = h + MoE(RMSNorm(h)) (moe_forward_block); "
+                        "dense: the dense SwiGLU FFN d -> 18432 -> d at the workload's T (moe_dense_ffn)")
     args = p.parse_args()
-    if args.op == "block" and args.impl == "reference":
+    if args.op != "layer" and args.impl == "reference":
         p.error("the reference arm times the layer")
     wl = WORKLOADS[args.workload]
     if args.tokens > 0:
         wl = wl.with_T(args.tokens)
     if args.impl == "reference":
         return run_reference(args, wl)
+    if args.op == "dense":
+        return run_dense(args, wl)
     return run_ours(args, wl)
 
 

@@ -84,6 +84,10 @@ def lib():
             L.moe_forward_block.restype = I
             L.moe_forward_block.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, ctypes.c_float,
                                             P, P, I, P, P, ctypes.c_size_t, P, P, P]
+            L.moe_dense_workspace_size.restype = ctypes.c_size_t
+            L.moe_dense_workspace_size.argtypes = [I, I, I, I, I]
+            L.moe_dense_ffn.restype = I
+            L.moe_dense_ffn.argtypes = [I, I, I, I, P, P, P, P, P, P, P, I, P, I, I, P, ctypes.c_size_t, P, P]
             L.moe_forward_plan.restype = I
             L.moe_forward_plan.argtypes = [ctypes.POINTER(MoeConfig), I, I, ctypes.c_void_p]
             L.moe_launch_count.restype = ctypes.c_ulonglong
@@ -286,6 +290,28 @@ def moe_forward_block(cfg: MoeConfig, weights, norm_g, h, bias, y, eps: float = 
                                    _p(y), _p(workspace), ws_bytes, _stream(stream),
                                    ctypes.byref(ev) if ev is not None else None,
                                    ctypes.byref(ro) if ro is not None else None), "moe_forward_block")
+
+
+def dense_workspace_size(d: int, hidden: int, act_dtype: int, weight_dtype: int, T: int) -> int:
+    return int(lib().moe_dense_workspace_size(int(d), int(hidden), int(act_dtype), int(weight_dtype), int(T)))
+
+
+def moe_dense_ffn(w_gate, w_up, w_down, x, y, s_gate=None, s_up=None, s_down=None, accumulate: bool = False,
+                  workspace=None, stream=None, stage_events=None):
+    """Dense SwiGLU FFN: y (+)= W_down(SiLU(W_gate x) * (W_up x)).  Weights bf16, or uint8 e4m3 codes with fp32
+    128x128 block scales s_*; x [T, d] bf16 (or fp32 for bf16 weights); y fp32 or bf16."""
+    for n, t in (("w_gate", w_gate), ("w_up", w_up), ("w_down", w_down), ("x", x), ("y", y),
+                 ("s_gate", s_gate), ("s_up", s_up), ("s_down", s_down), ("workspace", workspace)):
+        _dev(t, n)
+    hidden, d = w_gate.shape
+    wdt = MOE_E4M3 if w_gate.dtype == torch.uint8 else MOE_BF16
+    T = x.shape[0]
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    ev = _events(stage_events)
+    _check(lib().moe_dense_ffn(d, hidden, _dtype_code(x), wdt, _p(w_gate), _p(w_up), _p(w_down), _p(s_gate),
+                               _p(s_up), _p(s_down), _p(x), T, _p(y), _dtype_code(y), 1 if accumulate else 0,
+                               _p(workspace), ws_bytes, _stream(stream),
+                               ctypes.byref(ev) if ev is not None else None), "moe_dense_ffn")
 
 
 def moe_quantize_act(x, q, sx, stream=None):

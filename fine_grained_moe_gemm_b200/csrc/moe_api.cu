@@ -233,7 +233,9 @@ Plan make_plan(const moe_config* c, int T, int n_sm) {
     Plan p;
     p.fp8 = c->weight_dtype == MOE_E4M3;
     const int H = c->hidden, Hs = c->n_shared ? c->shared_hidden : c->hidden, d = c->d;
-    p.bn = pick_bn(((long long)T * c->top_k + c->n_experts - 1) / c->n_experts);
+    // token rows per group: the routed experts' average, or all T rows of the one
+    // dense group when there is no routed expert
+    p.bn = pick_bn(c->n_experts ? ((long long)T * c->top_k + c->n_experts - 1) / c->n_experts : T);
     // wide token tiles run on CTA pairs (2-SM MMA), each SM loading half of the
     // token rows.  bf16: 256 rows per item, 256 features per gate/up item, 512
     // rows per down item.  FP8: 128 rows per item (the promoted sums live in
@@ -294,6 +296,9 @@ moe_status forward_impl(const moe_config* cfg, const moe_weights* wt, const void
                         void* y, moe_dtype y_dtype, int accumulate, void* workspace, size_t ws_bytes,
                         moe_stream_t stream, const moe_stage_events* events, const moe_routing_out* routing,
                         const void* norm_g, float eps);
+moe_status run_experts(const moe_config* cfg, const moe_weights* wt, const Workspace& W, const Plan& plan,
+                       const DevInfo& di, int T, const void* x, bool act_quantised, void* y, moe_dtype y_dtype,
+                       int accumulate, const void* residual, cudaStream_t s, const moe_stage_events* events);
 
 }  // namespace
 
@@ -428,6 +433,82 @@ moe_status moe_rmsnorm(const void* h, const void* g, float eps, int T, int d, vo
                                       d, eps, static_cast<__nv_bfloat16*>(out), q, sx, (cudaStream_t)stream));
 }
 
+// The dense FFN runs as the layer's expert stages with no routed expert: one
+// group of all T rows in the always-on slot (hidden = the dense width).
+static moe_config dense_config(int d, int hidden, moe_dtype act_dtype, moe_dtype weight_dtype) {
+    moe_config c;
+    memset(&c, 0, sizeof(c));
+    c.d = d;
+    c.n_experts = 0;
+    c.n_groups = 1;
+    c.topk_groups = 1;
+    c.top_k = 0;
+    c.hidden = hidden;
+    c.n_shared = 1;
+    c.shared_hidden = hidden;
+    c.routed_scale = 1.0f;
+    c.act_dtype = act_dtype;
+    c.weight_dtype = weight_dtype;
+    return c;
+}
+
+static bool dense_shape_ok(int d, int hidden, moe_dtype act_dtype, moe_dtype weight_dtype) {
+    if (d <= 0 || hidden <= 0 || d % 128 || hidden % 128) return false;
+    if (act_dtype != MOE_F32 && act_dtype != MOE_BF16) return false;
+    if (weight_dtype != MOE_BF16 && weight_dtype != MOE_E4M3) return false;
+    return !(weight_dtype == MOE_E4M3 && act_dtype != MOE_BF16);
+}
+
+size_t moe_dense_workspace_size(int d, int hidden, moe_dtype act_dtype, moe_dtype weight_dtype, int T_max) {
+    if (!dense_shape_ok(d, hidden, act_dtype, weight_dtype) || T_max < 0) return 0;
+    const moe_config c = dense_config(d, hidden, act_dtype, weight_dtype);
+    return layout(&c, T_max, nullptr).bytes;
+}
+
+moe_status moe_dense_ffn(int d, int hidden, moe_dtype act_dtype, moe_dtype weight_dtype, const void* w_gate,
+                         const void* w_up, const void* w_down, const float* s_gate, const float* s_up,
+                         const float* s_down, const void* x, int T, void* y, moe_dtype y_dtype, int accumulate,
+                         void* workspace, size_t ws_bytes, moe_stream_t stream, const moe_stage_events* events) {
+    if (!dense_shape_ok(d, hidden, act_dtype, weight_dtype)) {
+        const bool bad_shape = d <= 0 || hidden <= 0 || d % 128 || hidden % 128;
+        return bad_shape ? MOE_ERR_INVALID_ARG : MOE_ERR_UNSUPPORTED;
+    }
+    if (T < 0 || (y_dtype != MOE_F32 && y_dtype != MOE_BF16) || (accumulate != 0 && accumulate != 1))
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    const bool fp8 = weight_dtype == MOE_E4M3;
+    if (!w_gate || !w_up || !w_down || !x || !y || !workspace) return MOE_ERR_INVALID_ARG;
+    if (fp8 && (!s_gate || !s_up || !s_down)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) || !aligned16(x) || !aligned16(y) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return MOE_ERR_INVALID_ARG;
+    const moe_config c = dense_config(d, hidden, act_dtype, weight_dtype);
+    if (ws_bytes < layout(&c, T, nullptr).bytes) return MOE_ERR_WORKSPACE;
+    DevInfo di;
+    moe_status st = check_device(&di);
+    if (st != MOE_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    moe_weights w;
+    memset(&w, 0, sizeof(w));
+    w.ws_gate = w_gate;
+    w.ws_up = w_up;
+    w.ws_down = w_down;
+    w.ss_gate = s_gate;
+    w.ss_up = s_up;
+    w.ss_down = s_down;
+    const Workspace W = layout(&c, T, workspace);
+    const Plan plan = make_plan(&c, T, di.sm_count);
+    const int mt_gu = plan.pair ? hidden / 256 : hidden / 128;
+    const int mt_dn = plan.pair ? d / 512 : (d + 255) / 256;
+    for (int i = 0; i < 2; ++i)  // no router: the first two stage marks coincide
+        if (events && events->ev[i]) cudaEventRecord((cudaEvent_t)events->ev[i], s);
+    if (launch_dense_schedule(T, plan.bn, mt_gu, mt_dn, W.row_off, W.item_gu, W.item_dn, W.row_tok, W.row_coef, s) !=
+        cudaSuccess)
+        return MOE_ERR_CUDA;
+    return run_experts(&c, &w, W, plan, di, T, x, false, y, y_dtype, accumulate, accumulate ? y : nullptr, s,
+                       events);
+}
+
 moe_status moe_forward_block(const moe_config* cfg, const moe_weights* wt, const void* norm_g, float eps,
                              const void* h, const float* bias, int T, void* y, void* workspace, size_t ws_bytes,
                              moe_stream_t stream, const moe_stage_events* events, const moe_routing_out* routing) {
@@ -444,6 +525,143 @@ moe_status moe_forward_block(const moe_config* cfg, const moe_weights* wt, const
 }  // extern "C"
 
 namespace {
+
+// Stages (3b)-(5) of the layer on tables the caller has built: the gather of
+// the activations in group order (FP8: quantised first unless act_quantised),
+// the gate/up and down grouped GEMMs, the combine and the output cast.  Used by
+// the MoE forward (groups = routed experts + the shared one) and by the dense
+// FFN (one group of all T rows in the shared-expert slot, n_experts = 0).
+moe_status run_experts(const moe_config* cfg, const moe_weights* wt, const Workspace& W, const Plan& plan,
+                       const DevInfo& di, int T, const void* x, bool act_quantised, void* y, moe_dtype y_dtype,
+                       int accumulate, const void* residual, cudaStream_t s, const moe_stage_events* events) {
+    const bool fp8 = cfg->weight_dtype == MOE_E4M3;
+    const int E = cfg->n_experts, k = cfg->top_k, d = cfg->d, H = cfg->hidden;
+    const int Hs = cfg->n_shared ? cfg->shared_hidden : H;
+    const int NG = E + cfg->n_shared;
+    const int rows_max = T * k + cfg->n_shared * T;
+    const int ldh = H > Hs ? H : Hs;
+    const int bn = plan.bn;
+    const bool pair = plan.pair, pair8 = plan.pair8;
+    const int box_rows = (pair || pair8) ? kPairBoxRows : kBoxRows;
+    const int mt_dn = pair ? d / 512 : (d + 255) / 256;
+    auto mark = [&](int i) {
+        if (events && events->ev[i]) cudaEventRecord((cudaEvent_t)events->ev[i], s);
+    };
+    if (fp8) {
+        if ((!act_quantised && launch_quant_act(static_cast<const __nv_bfloat16*>(x), T, d, W.x_q, W.sx, s) != cudaSuccess) ||
+            launch_gather_fp8(W.x_q, W.sx, d, W.row_tok, W.row_off + NG, rows_max, W.xq_perm, W.sxT, di.sm_count,
+                              s) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    } else if (launch_gather(x, cfg->act_dtype == MOE_F32, d, W.row_tok, W.row_off + NG, rows_max, W.x_perm,
+                             di.sm_count, s) != cudaSuccess) {
+        return MOE_ERR_CUDA;
+    }
+    mark(2);
+
+    // (4) gate/up grouped GEMM with the SwiGLU epilogue -> h_perm
+    auto wmap = [&](CUtensorMap* m, const void* p, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+        return fp8 ? map_u8(m, p, rows, cols, box_rows) : map_bf16(m, p, rows, cols, box_rows);
+    };
+    GemmArgs g;
+    memset(&g, 0, sizeof(g));
+    // weight rows per TMA box: the FP8 pair kernel stacks 64 gate over 64 up rows per CTA
+    const uint32_t gu_box = pair8 ? 64 : 128;
+    if (E && (!wmap(&g.a0, wt->w_gate, (uint64_t)E * H, d, gu_box) ||
+              !wmap(&g.a1, wt->w_up, (uint64_t)E * H, d, gu_box)))
+        return MOE_ERR_CUDA;
+    if (cfg->n_shared) {
+        if (!wmap(&g.s0, wt->ws_gate, Hs, d, gu_box) || !wmap(&g.s1, wt->ws_up, Hs, d, gu_box)) return MOE_ERR_CUDA;
+        if (!E) {
+            g.a0 = g.s0;
+            g.a1 = g.s1;
+        }
+    } else {
+        g.s0 = g.a0;
+        g.s1 = g.a1;
+    }
+    if (!(fp8 ? map_u8(&g.b, W.xq_perm, rows_max, d, box_rows) : map_bf16(&g.b, W.x_perm, rows_max, d, box_rows)))
+        return MOE_ERR_CUDA;
+    g.item_off = W.item_gu;
+    g.row_off = W.row_off;
+    g.n_groups = NG;
+    g.n_routed = E;
+    g.K_routed = g.K_shared = d;
+    g.mt_routed = pair ? H / 256 : H / 128;
+    g.mt_shared = pair ? Hs / 256 : Hs / 128;
+    g.rows_per_expert = H;
+    g.h = W.h_perm;
+    g.ldh = ldh;
+    if (fp8) {
+        g.sa0 = E ? wt->s_gate : wt->ss_gate;
+        g.sa1 = E ? wt->s_up : wt->ss_up;
+        g.ss0 = cfg->n_shared ? wt->ss_gate : wt->s_gate;
+        g.ss1 = cfg->n_shared ? wt->ss_up : wt->s_up;
+        g.a_rb_routed = H / 128;
+        g.a_rb_shared = Hs / 128;
+        g.sbT = W.sxT;
+        g.sb_ld = rows_max;
+        g.hq = W.hq;
+        g.hsT = W.shT;
+        g.hs_ld = rows_max;
+    }
+    const cudaError_t egu = pair8  ? launch_gemm2_fp8(MODE_GATEUP, &g, di.sm_count, s)
+                            : fp8  ? launch_gemm_fp8(MODE_GATEUP, bn, &g, di.sm_count, s)
+                            : pair ? launch_gemm2(MODE_GATEUP, &g, di.sm_count, s)
+                                   : launch_gemm(MODE_GATEUP, bn, &g, di.sm_count, s);
+    if (egu != cudaSuccess) return MOE_ERR_CUDA;
+    mark(3);
+
+    // (5) down GEMM, routing-weight scale and un-permute scatter into fp32
+    float* yacc = y_dtype == MOE_F32 ? static_cast<float*>(y) : W.y_acc;
+    if ((y_dtype == MOE_BF16 || !accumulate) &&
+        cudaMemsetAsync(yacc, 0, (size_t)T * d * sizeof(float), s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    GemmArgs dn;
+    memset(&dn, 0, sizeof(dn));
+    if (E && !wmap(&dn.a0, wt->w_down, (uint64_t)E * d, H, 128)) return MOE_ERR_CUDA;
+    if (cfg->n_shared) {
+        if (!wmap(&dn.s0, wt->ws_down, d, Hs, 128)) return MOE_ERR_CUDA;
+        if (!E) dn.a0 = dn.s0;
+    } else {
+        dn.s0 = dn.a0;
+    }
+    dn.a1 = dn.a0;
+    dn.s1 = dn.s0;
+    if (!(fp8 ? map_u8(&dn.b, W.hq, rows_max, ldh, box_rows) : map_bf16(&dn.b, W.h_perm, rows_max, ldh, box_rows)))
+        return MOE_ERR_CUDA;
+    dn.item_off = W.item_dn;
+    dn.row_off = W.row_off;
+    dn.n_groups = NG;
+    dn.n_routed = E;
+    dn.K_routed = H;
+    dn.K_shared = Hs;
+    dn.mt_routed = dn.mt_shared = mt_dn;
+    dn.rows_per_expert = d;
+    dn.y = yacc;
+    dn.row_coef = W.row_coef;
+    dn.row_tok = W.row_tok;
+    dn.ldy = d;
+    if (fp8) {
+        dn.sa0 = dn.sa1 = E ? wt->s_down : wt->ss_down;
+        dn.ss0 = dn.ss1 = cfg->n_shared ? wt->ss_down : wt->s_down;
+        dn.a_rb_routed = dn.a_rb_shared = d / 128;
+        dn.sbT = W.shT;
+        dn.sb_ld = rows_max;
+    }
+    const cudaError_t edn = pair8  ? launch_gemm2_fp8(MODE_DOWN, &dn, di.sm_count, s)
+                            : fp8  ? launch_gemm_fp8(MODE_DOWN, bn, &dn, di.sm_count, s)
+                            : pair ? launch_gemm2(MODE_DOWN, &dn, di.sm_count, s)
+                                   : launch_gemm(MODE_DOWN, bn, &dn, di.sm_count, s);
+    if (edn != cudaSuccess) return MOE_ERR_CUDA;
+    mark(4);
+
+    if (y_dtype == MOE_BF16 &&
+        launch_finalize_bf16(W.y_acc, static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(y),
+                             (size_t)T * d, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    mark(5);
+    return MOE_OK;
+}
 
 moe_status forward_impl(const moe_config* cfg, const moe_weights* wt, const void* x, const float* bias, int T,
                         void* y, moe_dtype y_dtype, int accumulate, void* workspace, size_t ws_bytes,
@@ -495,13 +713,9 @@ moe_status forward_impl(const moe_config* cfg, const moe_weights* wt, const void
     }
     const int E = cfg->n_experts, k = cfg->top_k, d = cfg->d, H = cfg->hidden;
     const int Hs = cfg->n_shared ? cfg->shared_hidden : H;
-    const int NG = E + cfg->n_shared;
-    const int rows_max = T * k + cfg->n_shared * T;
-    const int ldh = H > Hs ? H : Hs;
     const Plan plan = make_plan(cfg, T, di.sm_count);
     const int bn = plan.bn;
-    const bool pair = plan.pair, pair8 = plan.pair8;
-    const int box_rows = (pair || pair8) ? kPairBoxRows : kBoxRows;
+    const bool pair = plan.pair;
 
     auto mark = [&](int i) {
         if (events && events->ev[i]) cudaEventRecord((cudaEvent_t)events->ev[i], s);
@@ -548,114 +762,7 @@ moe_status forward_impl(const moe_config* cfg, const moe_weights* wt, const void
     pa.mt_dn = pair ? d / 512 : (d + 255) / 256;  // pair8: 256 down rows per item, as the 1-CTA kernels
     const cudaError_t ep = plan.permute_multi ? launch_permute_multi(pa, W.hist, s) : launch_permute(pa, s);
     if (ep != cudaSuccess) return MOE_ERR_CUDA;
-    if (fp8) {
-        if ((!norm_g && launch_quant_act(static_cast<const __nv_bfloat16*>(x), T, d, W.x_q, W.sx, s) != cudaSuccess) ||
-            launch_gather_fp8(W.x_q, W.sx, d, W.row_tok, W.row_off + NG, rows_max, W.xq_perm, W.sxT, di.sm_count,
-                              s) != cudaSuccess)
-            return MOE_ERR_CUDA;
-    } else if (launch_gather(x, cfg->act_dtype == MOE_F32, d, W.row_tok, W.row_off + NG, rows_max, W.x_perm,
-                             di.sm_count, s) != cudaSuccess) {
-        return MOE_ERR_CUDA;
-    }
-    mark(2);
-
-    // (4) gate/up grouped GEMM with the SwiGLU epilogue -> h_perm
-    auto wmap = [&](CUtensorMap* m, const void* p, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-        return fp8 ? map_u8(m, p, rows, cols, box_rows) : map_bf16(m, p, rows, cols, box_rows);
-    };
-    GemmArgs g;
-    memset(&g, 0, sizeof(g));
-    // weight rows per TMA box: the FP8 pair kernel stacks 64 gate over 64 up rows per CTA
-    const uint32_t gu_box = pair8 ? 64 : 128;
-    if (!wmap(&g.a0, wt->w_gate, (uint64_t)E * H, d, gu_box) || !wmap(&g.a1, wt->w_up, (uint64_t)E * H, d, gu_box))
-        return MOE_ERR_CUDA;
-    if (cfg->n_shared) {
-        if (!wmap(&g.s0, wt->ws_gate, Hs, d, gu_box) || !wmap(&g.s1, wt->ws_up, Hs, d, gu_box)) return MOE_ERR_CUDA;
-    } else {
-        g.s0 = g.a0;
-        g.s1 = g.a1;
-    }
-    if (!(fp8 ? map_u8(&g.b, W.xq_perm, rows_max, d, box_rows) : map_bf16(&g.b, W.x_perm, rows_max, d, box_rows)))
-        return MOE_ERR_CUDA;
-    g.item_off = W.item_gu;
-    g.row_off = W.row_off;
-    g.n_groups = NG;
-    g.n_routed = E;
-    g.K_routed = g.K_shared = d;
-    g.mt_routed = pa.mt_gu_routed;
-    g.mt_shared = pa.mt_gu_shared;
-    g.rows_per_expert = H;
-    g.h = W.h_perm;
-    g.ldh = ldh;
-    if (fp8) {
-        g.sa0 = wt->s_gate;
-        g.sa1 = wt->s_up;
-        g.ss0 = cfg->n_shared ? wt->ss_gate : wt->s_gate;
-        g.ss1 = cfg->n_shared ? wt->ss_up : wt->s_up;
-        g.a_rb_routed = H / 128;
-        g.a_rb_shared = Hs / 128;
-        g.sbT = W.sxT;
-        g.sb_ld = rows_max;
-        g.hq = W.hq;
-        g.hsT = W.shT;
-        g.hs_ld = rows_max;
-    }
-    const cudaError_t egu = pair8  ? launch_gemm2_fp8(MODE_GATEUP, &g, di.sm_count, s)
-                            : fp8  ? launch_gemm_fp8(MODE_GATEUP, bn, &g, di.sm_count, s)
-                            : pair ? launch_gemm2(MODE_GATEUP, &g, di.sm_count, s)
-                                   : launch_gemm(MODE_GATEUP, bn, &g, di.sm_count, s);
-    if (egu != cudaSuccess) return MOE_ERR_CUDA;
-    mark(3);
-
-    // (5) down GEMM, routing-weight scale and un-permute scatter into fp32
-    float* yacc = y_dtype == MOE_F32 ? static_cast<float*>(y) : W.y_acc;
-    if ((y_dtype == MOE_BF16 || !accumulate) &&
-        cudaMemsetAsync(yacc, 0, (size_t)T * d * sizeof(float), s) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    GemmArgs dn;
-    memset(&dn, 0, sizeof(dn));
-    if (!wmap(&dn.a0, wt->w_down, (uint64_t)E * d, H, 128)) return MOE_ERR_CUDA;
-    if (cfg->n_shared) {
-        if (!wmap(&dn.s0, wt->ws_down, d, Hs, 128)) return MOE_ERR_CUDA;
-    } else {
-        dn.s0 = dn.a0;
-    }
-    dn.a1 = dn.a0;
-    dn.s1 = dn.s0;
-    if (!(fp8 ? map_u8(&dn.b, W.hq, rows_max, ldh, box_rows) : map_bf16(&dn.b, W.h_perm, rows_max, ldh, box_rows)))
-        return MOE_ERR_CUDA;
-    dn.item_off = W.item_dn;
-    dn.row_off = W.row_off;
-    dn.n_groups = NG;
-    dn.n_routed = E;
-    dn.K_routed = H;
-    dn.K_shared = Hs;
-    dn.mt_routed = dn.mt_shared = pa.mt_dn;
-    dn.rows_per_expert = d;
-    dn.y = yacc;
-    dn.row_coef = W.row_coef;
-    dn.row_tok = W.row_tok;
-    dn.ldy = d;
-    if (fp8) {
-        dn.sa0 = dn.sa1 = wt->s_down;
-        dn.ss0 = dn.ss1 = cfg->n_shared ? wt->ss_down : wt->s_down;
-        dn.a_rb_routed = dn.a_rb_shared = d / 128;
-        dn.sbT = W.shT;
-        dn.sb_ld = rows_max;
-    }
-    const cudaError_t edn = pair8  ? launch_gemm2_fp8(MODE_DOWN, &dn, di.sm_count, s)
-                            : fp8  ? launch_gemm_fp8(MODE_DOWN, bn, &dn, di.sm_count, s)
-                            : pair ? launch_gemm2(MODE_DOWN, &dn, di.sm_count, s)
-                                   : launch_gemm(MODE_DOWN, bn, &dn, di.sm_count, s);
-    if (edn != cudaSuccess) return MOE_ERR_CUDA;
-    mark(4);
-
-    if (y_dtype == MOE_BF16 &&
-        launch_finalize_bf16(W.y_acc, static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(y),
-                             (size_t)T * d, s) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    mark(5);
-    return MOE_OK;
+    return run_experts(cfg, wt, W, plan, di, T, x, norm_g != nullptr, y, y_dtype, accumulate, residual, s, events);
 }
 
 }  // namespace

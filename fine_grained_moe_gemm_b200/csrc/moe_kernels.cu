@@ -14,6 +14,7 @@
 //   moe_gemm2_fp8_kernel  CTA-pair e4m3 GEMM (moe_gemm2_fp8.cuh)
 //   update_bias_kernel    selection-bias controller step
 //   rmsnorm_kernel        pre-norm of the sublayer (+ the 1x128 e4m3 quantisation)
+//   dense_schedule_kernel the one-group tables of the dense FFN
 //   finalize_kernel       fp32 combine buffer -> bf16 output (+ residual)
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -502,6 +503,31 @@ __global__ void __launch_bounds__(256) gather_fp8_kernel(const uint8_t* __restri
     }
 }
 
+// ============================================================================ dense schedule
+// The tables of one group of all T rows (the dense FFN): row_tok = identity,
+// row_coef = 1, group extents {0, T}, tile counts of the two GEMMs.
+__global__ void __launch_bounds__(256) dense_schedule_kernel(int T, int bn, int mt_gu, int mt_dn,
+                                                             int32_t* __restrict__ row_off,
+                                                             int32_t* __restrict__ item_gu,
+                                                             int32_t* __restrict__ item_dn,
+                                                             int32_t* __restrict__ row_tok,
+                                                             float* __restrict__ row_coef) {
+    const int i0 = blockIdx.x * blockDim.x + threadIdx.x;
+    for (int r = i0; r < T; r += gridDim.x * blockDim.x) {
+        row_tok[r] = r;
+        row_coef[r] = 1.0f;
+    }
+    if (i0 == 0) {
+        const int chunks = (T + bn - 1) / bn;
+        row_off[0] = 0;
+        row_off[1] = T;
+        item_gu[0] = 0;
+        item_gu[1] = chunks * mt_gu;
+        item_dn[0] = 0;
+        item_dn[1] = chunks * mt_dn;
+    }
+}
+
 // ============================================================================ pre-norm
 // "RMSNorm" box: r = 1/sqrt(mean_c h[c]^2 + eps), the mean reduced in fp32;
 // out = bf16(bf16(h * r) * g).  With q and sx the same pass also writes the
@@ -881,6 +907,16 @@ cudaError_t launch_finalize_bf16(const float* acc, const __nv_bfloat16* residual
     if (grid < 1) grid = 1;
     note_launch();
     finalize_kernel<<<(unsigned)grid, 256, 0, s>>>(acc, residual, y, n8);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dense_schedule(int T, int bn, int mt_gu, int mt_dn, int32_t* row_off, int32_t* item_gu,
+                                  int32_t* item_dn, int32_t* row_tok, float* row_coef, cudaStream_t s) {
+    int grid = (T + 255) / 256;
+    if (grid > 148) grid = 148;
+    if (grid < 1) grid = 1;
+    note_launch();
+    dense_schedule_kernel<<<grid, 256, 0, s>>>(T, bn, mt_gu, mt_dn, row_off, item_gu, item_dn, row_tok, row_coef);
     return cudaGetLastError();
 }
 

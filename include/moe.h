@@ -267,6 +267,27 @@ MOE_API moe_status moe_forward_block(const moe_config* cfg, const moe_weights* w
                                      size_t ws_bytes, moe_stream_t stream, const moe_stage_events* events,
                                      const moe_routing_out* routing);
 
+/* Dense SwiGLU FFN ("DeepSeek-V3" llm-vis, "SwiGLU MLP" box; the model's first
+ * layers use a dense FFN of hidden width 18432 in place of the experts):
+ *   y (+)= W_down ( SiLU(W_gate x) * (W_up x) )
+ * on the same grouped-GEMM kernels as the experts (one group of all T rows).
+ * w_gate, w_up: [hidden, d]; w_down: [d, hidden] (nn.Linear layout), bf16, or
+ * e4m3 codes with s_gate, s_up [hidden/128, d/128] and s_down [d/128, hidden/128]
+ * fp32 block scales (weight_dtype MOE_E4M3; x is then quantised per 1x128 tile
+ * and h stored as e4m3 with 1x128 scales, as in the FP8 layer).  x: [T, d]
+ * (MOE_BF16, or MOE_F32 rounded to bf16; FP8 needs bf16); y: [T, d] fp32 or
+ * bf16, `accumulate` adds into it.  d and hidden multiples of 128.  h is
+ * stored in bf16 between the projections.  workspace: moe_dense_workspace_size
+ * bytes, 256-byte aligned.  events (optional) as in moe_forward_ex: ev[0] = ev[1]
+ * (no router), ev[2] after the table setup and the gather.  Errors as
+ * moe_forward. */
+MOE_API size_t moe_dense_workspace_size(int d, int hidden, moe_dtype act_dtype, moe_dtype weight_dtype, int T_max);
+MOE_API moe_status moe_dense_ffn(int d, int hidden, moe_dtype act_dtype, moe_dtype weight_dtype, const void* w_gate,
+                                 const void* w_up, const void* w_down, const float* s_gate, const float* s_up,
+                                 const float* s_down, const void* x, int T, void* y, moe_dtype y_dtype,
+                                 int accumulate, void* workspace, size_t ws_bytes, moe_stream_t stream,
+                                 const moe_stage_events* events);
+
 /* Size of the device scratch array that moe_forward_noalloc uses in place of
  * a caller-provided workspace: 32 MiB.  At the DeepSeek-V3 sizes (d = 7168,
  * 256 experts, top-8, H = Hs = 2048, one shared expert) that holds up to

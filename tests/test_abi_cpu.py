@@ -126,3 +126,20 @@ def test_prenorm_and_block_arguments(L):
     assert blk(cfg, P(20), 1 << 30) == moe.MOE_ERR_INVALID_ARG         # misaligned gain
     f32 = cfg_of(WORKLOADS["tiny"])                                     # fp32 activations: not a bf16 stream
     assert blk(f32, P(16), 1 << 30) == moe.MOE_ERR_UNSUPPORTED
+
+
+def test_dense_arguments(L):
+    P = ctypes.c_void_p
+    B, F, E8 = moe.MOE_BF16, moe.MOE_F32, moe.MOE_E4M3
+    assert moe.dense_workspace_size(7168, 18432, B, B, 128) > 128 * 18432 * 2
+    assert moe.dense_workspace_size(7168, 100, B, B, 128) == 0          # hidden not a multiple of 128
+    assert moe.dense_workspace_size(7168, 18432, F, E8, 128) == 0       # FP8 needs bf16 activations
+    call = lambda d, h, act, wdt, ws: L.moe_dense_ffn(d, h, act, wdt, P(16), P(16), P(16), P(16), P(16), P(16),
+                                                      P(16), 4, P(16), B, 0, P(1024), ws, None, None)
+    assert call(7168, 100, B, B, 1 << 30) == moe.MOE_ERR_INVALID_ARG
+    assert call(7168, 18432, F, E8, 1 << 30) == moe.MOE_ERR_UNSUPPORTED
+    assert call(7168, 18432, B, B, 1024) == moe.MOE_ERR_WORKSPACE
+    assert L.moe_dense_ffn(7168, 18432, B, E8, P(16), P(16), P(16), None, None, None, P(16), 4, P(16), B, 0,
+                           P(1024), 1 << 30, None, None) == moe.MOE_ERR_INVALID_ARG   # FP8 without scales
+    assert L.moe_dense_ffn(7168, 18432, B, B, None, None, None, None, None, None, None, 0, None, B, 0, None, 0,
+                           None, None) == moe.MOE_OK                          # T = 0

@@ -211,6 +211,22 @@ def make_weights(wl: Workload, device="cpu", seed: int = 0) -> dict:
     return W
 
 
+DENSE_HIDDEN = 18432  # the dense FFN width of the model's first layers ("At a glance" table)
+DENSE_WID = 20       # generator stream of the dense FFN weights
+
+
+def make_dense_weights(d: int, hidden: int, fp8: bool, device="cpu", seed: int = 0) -> dict:
+    """Dense SwiGLU FFN weights w_gate/w_up [hidden, d], w_down [d, hidden], bf16 N(0, 0.02);
+    with fp8 the e4m3 codes (uint8) plus fp32 128x128 block scales s_gate/s_up/s_down."""
+    W = {}
+    for name, shape in (("w_gate", (hidden, d)), ("w_up", (hidden, d)), ("w_down", (d, hidden))):
+        W[name] = _normal_bf16(shape, WEIGHT_STD, device, _seed(seed, DENSE_WID + d % 7, name, hidden))
+    if fp8:
+        for name in ("w_gate", "w_up", "w_down"):
+            W[name], W["s" + name[1:]] = _quantise_blocks_e4m3(W[name])
+    return W
+
+
 def make_inputs(wl: Workload, device="cpu", seed: int = 0, T: int | None = None) -> dict:
     """Weights, x and bias of one workload on ``device``."""
     W = make_weights(wl, device, seed)
