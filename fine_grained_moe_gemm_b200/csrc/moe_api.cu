@@ -298,7 +298,8 @@ moe_status forward_impl(const moe_config* cfg, const moe_weights* wt, const void
                         const void* norm_g, float eps);
 moe_status run_experts(const moe_config* cfg, const moe_weights* wt, const Workspace& W, const Plan& plan,
                        const DevInfo& di, int T, const void* x, bool act_quantised, void* y, moe_dtype y_dtype,
-                       int accumulate, const void* residual, cudaStream_t s, const moe_stage_events* events);
+                       int accumulate, const void* residual, cudaStream_t s, const moe_stage_events* events,
+                       int dn_splits);
 
 }  // namespace
 
@@ -500,13 +501,25 @@ moe_status moe_dense_ffn(int d, int hidden, moe_dtype act_dtype, moe_dtype weigh
     const Plan plan = make_plan(&c, T, di.sm_count);
     const int mt_gu = plan.pair ? hidden / 256 : hidden / 128;
     const int mt_dn = plan.pair ? d / 512 : (d + 255) / 256;
+    // a few token chunks leave most SMs without a down tile (d / 512 = 14 pair tiles at
+    // d = 7168): split the long K (= hidden) of the down GEMM so that one wave fills the
+    // GPU; the splits add into y by the combine's atomics.  bf16 kernels only.
+    int dn_splits = 1;
+    if (!plan.fp8) {
+        const int units = plan.pair ? di.sm_count / 2 : di.sm_count;
+        const int tiles = ((T + plan.bn - 1) / plan.bn) * mt_dn;
+        const int max_splits = hidden / 64 / 4;  // at least four 64-wide K blocks a split
+        if (tiles < units) dn_splits = units / tiles;
+        if (dn_splits > max_splits) dn_splits = max_splits;
+        if (dn_splits < 1) dn_splits = 1;
+    }
     for (int i = 0; i < 2; ++i)  // no router: the first two stage marks coincide
         if (events && events->ev[i]) cudaEventRecord((cudaEvent_t)events->ev[i], s);
-    if (launch_dense_schedule(T, plan.bn, mt_gu, mt_dn, W.row_off, W.item_gu, W.item_dn, W.row_tok, W.row_coef, s) !=
-        cudaSuccess)
+    if (launch_dense_schedule(T, plan.bn, mt_gu, mt_dn * dn_splits, W.row_off, W.item_gu, W.item_dn, W.row_tok,
+                              W.row_coef, s) != cudaSuccess)
         return MOE_ERR_CUDA;
     return run_experts(&c, &w, W, plan, di, T, x, false, y, y_dtype, accumulate, accumulate ? y : nullptr, s,
-                       events);
+                       events, dn_splits);
 }
 
 moe_status moe_forward_block(const moe_config* cfg, const moe_weights* wt, const void* norm_g, float eps,
@@ -533,7 +546,8 @@ namespace {
 // FFN (one group of all T rows in the shared-expert slot, n_experts = 0).
 moe_status run_experts(const moe_config* cfg, const moe_weights* wt, const Workspace& W, const Plan& plan,
                        const DevInfo& di, int T, const void* x, bool act_quantised, void* y, moe_dtype y_dtype,
-                       int accumulate, const void* residual, cudaStream_t s, const moe_stage_events* events) {
+                       int accumulate, const void* residual, cudaStream_t s, const moe_stage_events* events,
+                       int dn_splits) {
     const bool fp8 = cfg->weight_dtype == MOE_E4M3;
     const int E = cfg->n_experts, k = cfg->top_k, d = cfg->d, H = cfg->hidden;
     const int Hs = cfg->n_shared ? cfg->shared_hidden : H;
@@ -636,6 +650,7 @@ moe_status run_experts(const moe_config* cfg, const moe_weights* wt, const Works
     dn.K_routed = H;
     dn.K_shared = Hs;
     dn.mt_routed = dn.mt_shared = mt_dn;
+    dn.k_splits = dn_splits;  // bf16 kernels only: the tables count mt_dn * dn_splits tiles per chunk
     dn.rows_per_expert = d;
     dn.y = yacc;
     dn.row_coef = W.row_coef;
@@ -762,7 +777,7 @@ moe_status forward_impl(const moe_config* cfg, const moe_weights* wt, const void
     pa.mt_dn = pair ? d / 512 : (d + 255) / 256;  // pair8: 256 down rows per item, as the 1-CTA kernels
     const cudaError_t ep = plan.permute_multi ? launch_permute_multi(pa, W.hist, s) : launch_permute(pa, s);
     if (ep != cudaSuccess) return MOE_ERR_CUDA;
-    return run_experts(cfg, wt, W, plan, di, T, x, norm_g != nullptr, y, y_dtype, accumulate, residual, s, events);
+    return run_experts(cfg, wt, W, plan, di, T, x, norm_g != nullptr, y, y_dtype, accumulate, residual, s, events, 1);
 }
 
 }  // namespace

@@ -102,14 +102,17 @@ __device__ __forceinline__ Item decode_item(const GemmArgs& P, int i) {
         else hi = mid - 1;
     }
     it.g = lo;
-    it.split = 0;
-    it.n_splits = 1;
+    // k_splits > 1 (DOWN of a schedule with few tiles): each (tile, split) pair is one
+    // item; the splits of a tile add their partial sums into y by the same atomics
+    it.n_splits = P.k_splits > 1 ? P.k_splits : 1;
     int local = i - __ldg(&P.item_off[lo]);
     int r0 = __ldg(&P.row_off[lo]);
     int ng = __ldg(&P.row_off[lo + 1]) - r0;
     int nch = (ng + BN - 1) / BN;
-    it.m = local / nch;
-    int c = local - it.m * nch;
+    const int ms = local / nch;  // tile-major, split, then token chunk (chunks of a weight slice run together)
+    it.m = ms / it.n_splits;
+    it.split = ms - it.m * it.n_splits;
+    int c = local - ms * nch;
     it.row0 = r0 + c * BN;
     it.nvalid = min(BN, ng - c * BN);
     it.shared = lo >= P.n_routed;

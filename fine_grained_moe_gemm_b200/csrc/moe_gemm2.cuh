@@ -210,7 +210,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
                 }
                 const int brow = it.row0 + (int)rank * nh;
                 bool ok = true;
-                for (int kb = 0; kb < KB; ++kb) {
+                for (int kb = item_kb0(it, KB); kb < item_kb1(it, KB); ++kb) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
                     uint8_t* sa = ring + stage * C::STAGE_BYTES;
                     uint8_t* sb = sa + C::A_BYTES;
@@ -243,7 +243,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
                 const uint32_t d0 = tmem_base;
                 const uint32_t d1 = tmem_base + PAIR_BN;
                 bool ok = true;
-                for (int kb = 0; kb < KB; ++kb) {
+                const int kb0 = item_kb0(it, KB), kb1 = item_kb1(it, KB);
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait_bounded(&full[stage], phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(ring + stage * C::STAGE_BYTES);
@@ -252,7 +253,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
                     const uint64_t bdesc = smem_desc_sw128(a_addr + C::A_BYTES);
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const uint32_t accum = (kb | k) != 0 ? 1u : 0u;
+                        const uint32_t accum = (kb > kb0 || k != 0) ? 1u : 0u;
                         mma2_bf16(d0, adesc0 + 2ull * k, bdesc + 2ull * k, idesc, accum);
                         mma2_bf16(d1, adesc1 + 2ull * k, bdesc + 2ull * k, idesc, accum);
                     }

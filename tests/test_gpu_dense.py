@@ -59,7 +59,7 @@ def reference(W, x, tokens):
                             x_is_f32=x.dtype == torch.float32, **kw)
 
 
-@pytest.mark.parametrize("d,hidden,T", [(256, 512, 64), (256, 512, 1), (256, 512, 300), (512, 256, 300),
+@pytest.mark.parametrize("d,hidden,T", [(256, 512, 64), (256, 512, 1), (256, 512, 300), (512, 256, 300), (512, 2048, 100),
                                         (256, 384, 1000)])
 def test_dense_small_full(d, hidden, T):
     W = weights(d, hidden, False)
