@@ -90,6 +90,8 @@ def lib():
             L.moe_dense_ffn.argtypes = [I, I, I, I, P, P, P, P, P, P, P, I, P, I, I, P, ctypes.c_size_t, P, P]
             L.moe_forward_plan.restype = I
             L.moe_forward_plan.argtypes = [ctypes.POINTER(MoeConfig), I, I, ctypes.c_void_p]
+            L.moe_selftest_wait_timeout.restype = I
+            L.moe_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, P]
             L.moe_launch_count.restype = ctypes.c_ulonglong
             L.moe_launch_count.argtypes = []
             L.moe_update_bias.restype = I
@@ -244,6 +246,12 @@ def moe_forward(cfg: MoeConfig, weights, x, bias, y, accumulate: bool = False, w
                                 1 if accumulate else 0, _p(workspace), ws_bytes, _stream(stream),
                                 ctypes.byref(ev) if ev is not None else None,
                                 ctypes.byref(ro) if ro is not None else None), "moe_forward")
+
+
+def selftest_wait_timeout(limit_ns: int = 1_000_000, stream=None):
+    """Launches a kernel whose bounded wait runs out after limit_ns; the device error word then holds
+    MOE_DEVERR_TIMEOUT."""
+    _check(lib().moe_selftest_wait_timeout(int(limit_ns), _stream(stream)), "moe_selftest_wait_timeout")
 
 
 def launch_count() -> int:

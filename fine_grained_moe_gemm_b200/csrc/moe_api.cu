@@ -350,6 +350,14 @@ moe_status moe_quantize_act(const void* x, int T, int d, uint8_t* q, float* sx, 
 
 unsigned long long moe_launch_count(void) { return launch_count(); }
 
+moe_status moe_selftest_wait_timeout(unsigned long long limit_ns, moe_stream_t stream) {
+    if (limit_ns == 0 || limit_ns > 1000000000ull) return MOE_ERR_INVALID_ARG;
+    DevInfo di;
+    moe_status st = check_device(&di);
+    if (st != MOE_OK) return st;
+    return cuda_status(launch_wait_selftest(limit_ns, (cudaStream_t)stream));
+}
+
 moe_status moe_forward_plan(const moe_config* cfg, int T, moe_dtype y_dtype, moe_plan* out) {
     moe_status st = check_config(cfg);
     if (st != MOE_OK) return st;

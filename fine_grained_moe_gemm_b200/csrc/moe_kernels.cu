@@ -503,6 +503,22 @@ __global__ void __launch_bounds__(256) gather_fp8_kernel(const uint8_t* __restri
     }
 }
 
+// ============================================================================ wait self-test
+// The failure path of the bounded waits, on its own: one thread waits on an
+// mbarrier that nothing completes; after limit_ns the wait gives up, sets
+// MOE_DEVERR_TIMEOUT and the kernel returns (no TMA, TMEM or MMA in flight).
+__global__ void __launch_bounds__(32) wait_selftest_kernel(unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait_bounded(&bar, 0, &abort_flag, limit_ns);
+}
+
 // ============================================================================ dense schedule
 // The tables of one group of all T rows (the dense FFN): row_tok = identity,
 // row_coef = 1, group extents {0, T}, tile counts of the two GEMMs.
@@ -917,6 +933,12 @@ cudaError_t launch_dense_schedule(int T, int bn, int mt_gu, int mt_dn, int32_t* 
     if (grid < 1) grid = 1;
     note_launch();
     dense_schedule_kernel<<<grid, 256, 0, s>>>(T, bn, mt_gu, mt_dn, row_off, item_gu, item_dn, row_tok, row_coef);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t s) {
+    note_launch();
+    wait_selftest_kernel<<<1, 32, 0, s>>>(limit_ns);
     return cudaGetLastError();
 }
 

@@ -105,6 +105,8 @@ cudaError_t launch_update_bias(const int32_t* counts, int E, float* bias, float 
 // y[i] = bf16(acc[i] (+ y[i]))
 cudaError_t launch_finalize_bf16(const float* acc, const __nv_bfloat16* residual, __nv_bfloat16* y, size_t n,
                                  cudaStream_t s);
+// a bounded mbarrier wait that runs out after limit_ns (sets MOE_DEVERR_TIMEOUT)
+cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t s);
 // dense FFN tables: one group of T rows, identity rows, coefficient 1
 cudaError_t launch_dense_schedule(int T, int bn, int mt_gu, int mt_dn, int32_t* row_off, int32_t* item_gu,
                                   int32_t* item_dn, int32_t* row_tok, float* row_coef, cudaStream_t s);

@@ -199,6 +199,12 @@ typedef struct moe_plan {
 } moe_plan;
 MOE_API moe_status moe_forward_plan(const moe_config* cfg, int T, moe_dtype y_dtype, moe_plan* plan);
 
+/* Self-test of the failure path every in-kernel wait has: one kernel waits on
+ * an mbarrier that nothing completes, gives up after limit_ns (at most 1 s)
+ * and sets MOE_DEVERR_TIMEOUT in the device error word (read it with
+ * moe_device_error); the context stays usable.  Nothing else runs in it. */
+MOE_API moe_status moe_selftest_wait_timeout(unsigned long long limit_ns, moe_stream_t stream);
+
 /* Number of kernels this library has launched in this process, over all
  * devices and streams (a diagnostic counter; never reset). */
 MOE_API unsigned long long moe_launch_count(void);

@@ -143,3 +143,8 @@ def test_dense_arguments(L):
                            P(1024), 1 << 30, None, None) == moe.MOE_ERR_INVALID_ARG   # FP8 without scales
     assert L.moe_dense_ffn(7168, 18432, B, B, None, None, None, None, None, None, None, 0, None, B, 0, None, 0,
                            None, None) == moe.MOE_OK                          # T = 0
+
+
+def test_selftest_arguments(L):
+    assert L.moe_selftest_wait_timeout(0, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_selftest_wait_timeout(2_000_000_000, None) == moe.MOE_ERR_INVALID_ARG
