@@ -124,6 +124,19 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
+// (a0, a1) += (p0, p1) * (s0, s1): two fp32 fused multiply-adds in one packed
+// instruction (sm_100), each rounded exactly as fmaf.
+__device__ __forceinline__ void fma2(float& a0, float& a1, float p0, float p1, float s0, float s1) {
+    asm("{\n\t.reg .b64 pa, pb, pc;\n\t"
+        "mov.b64 pa, {%2, %3};\n\t"
+        "mov.b64 pb, {%4, %5};\n\t"
+        "mov.b64 pc, {%0, %1};\n\t"
+        "fma.rn.f32x2 pc, pa, pb, pc;\n\t"
+        "mov.b64 {%0, %1}, pc;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(p0), "f"(p1), "f"(s0), "f"(s1));
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");

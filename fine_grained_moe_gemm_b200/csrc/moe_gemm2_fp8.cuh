@@ -285,16 +285,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
                     for (int j = 0; j < 32; j += 4) {
                         const float4 s0 = *reinterpret_cast<const float4*>(my_sc + j);
-                        acc[0][j + 0] = fmaf(p0[j + 0], s0.x, acc[0][j + 0]);
-                        acc[0][j + 1] = fmaf(p0[j + 1], s0.y, acc[0][j + 1]);
-                        acc[0][j + 2] = fmaf(p0[j + 2], s0.z, acc[0][j + 2]);
-                        acc[0][j + 3] = fmaf(p0[j + 3], s0.w, acc[0][j + 3]);
+                        fma2(acc[0][j + 0], acc[0][j + 1], p0[j + 0], p0[j + 1], s0.x, s0.y);
+                        fma2(acc[0][j + 2], acc[0][j + 3], p0[j + 2], p0[j + 3], s0.z, s0.w);
                         if (two) {
                             const float4 s1 = *reinterpret_cast<const float4*>(my_sc + 32 + j);
-                            acc[1][j + 0] = fmaf(p1[j + 0], s1.x, acc[1][j + 0]);
-                            acc[1][j + 1] = fmaf(p1[j + 1], s1.y, acc[1][j + 1]);
-                            acc[1][j + 2] = fmaf(p1[j + 2], s1.z, acc[1][j + 2]);
-                            acc[1][j + 3] = fmaf(p1[j + 3], s1.w, acc[1][j + 3]);
+                            fma2(acc[1][j + 0], acc[1][j + 1], p1[j + 0], p1[j + 1], s1.x, s1.y);
+                            fma2(acc[1][j + 2], acc[1][j + 3], p1[j + 2], p1[j + 3], s1.z, s1.w);
                         }
                     }
                     __syncwarp();
