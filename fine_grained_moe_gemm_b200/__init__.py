@@ -149,6 +149,20 @@ def _dev(t: torch.Tensor, name: str):
         raise ValueError(f"{name} must be a contiguous CUDA tensor")
 
 
+def _shape(t, name, shape, dtypes):
+    """The C ABI takes raw pointers: check here what it cannot (shape and element type)."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected one of {dtypes}")
+
+
+_ACT = {MOE_F32: (torch.float32,), MOE_BF16: (torch.bfloat16,)}
+_OUT = (torch.float32, torch.bfloat16)
+
+
 def workspace_size(cfg: MoeConfig, T: int) -> int:
     return int(lib().moe_workspace_size(ctypes.byref(cfg), int(T)))
 
@@ -159,6 +173,13 @@ def moe_route(cfg: MoeConfig, x, w_router, logits, bias, topk_idx, topk_w, strea
                  ("topk_w", topk_w)):
         _dev(t, n)
     T = logits.shape[0]
+    E, k = cfg.n_experts, cfg.top_k
+    _shape(x, "x", (T, cfg.d), _ACT.get(cfg.act_dtype, ()))
+    _shape(w_router, "w_router", (E, cfg.d), (torch.bfloat16,))
+    _shape(logits, "logits", (T, E), (torch.float32,))
+    _shape(bias, "bias", (E,), (torch.float32,))
+    _shape(topk_idx, "topk_idx", (T, k), (torch.int32,))
+    _shape(topk_w, "topk_w", (T, k), (torch.float32,))
     _check(lib().moe_route(ctypes.byref(cfg), _p(x), _p(w_router), _p(logits), _p(bias), T, _p(topk_idx),
                            _p(topk_w), _stream(stream)), "moe_route")
 
@@ -167,6 +188,13 @@ def moe_permute(cfg: MoeConfig, topk_idx, counts, offsets, src, inv, stream=None
     for n, t in (("topk_idx", topk_idx), ("counts", counts), ("offsets", offsets), ("src", src), ("inv", inv)):
         _dev(t, n)
     T = topk_idx.shape[0]
+    E, k = cfg.n_experts, cfg.top_k
+    _shape(topk_idx, "topk_idx", (T, k), (torch.int32,))
+    for n, t, shp in (("counts", counts, (E,)), ("offsets", offsets, (E + 1,))):
+        _shape(t, n, shp, (torch.int32,))
+    for n, t in (("src", src), ("inv", inv)):  # flat buffers of at least T * k entries
+        if t.dtype != torch.int32 or t.dim() != 1 or t.numel() < T * k:
+            raise ValueError(f"{n}: needs an int32 vector of at least {T * k} entries")
     _check(lib().moe_permute(ctypes.byref(cfg), _p(topk_idx), T, _p(counts), _p(offsets), _p(src), _p(inv),
                              _stream(stream)), "moe_permute")
 
@@ -240,6 +268,9 @@ def moe_forward(cfg: MoeConfig, weights, x, bias, y, accumulate: bool = False, w
         _dev(t, n)
     mw = weights if isinstance(weights, MoeWeights) else make_weights(weights)
     T = x.shape[0]
+    _shape(x, "x", (T, cfg.d), _ACT.get(cfg.act_dtype, ()))
+    _shape(bias, "bias", (cfg.n_experts,), (torch.float32,))
+    _shape(y, "y", (T, cfg.d), _OUT)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     ev, ro = _events(stage_events), _routing(routing_out)
     _check(lib().moe_forward_ex(ctypes.byref(cfg), ctypes.byref(mw), _p(x), _p(bias), T, _p(y), _dtype_code(y),
@@ -292,6 +323,10 @@ def moe_forward_block(cfg: MoeConfig, weights, norm_g, h, bias, y, eps: float = 
         _dev(t, n)
     mw = weights if isinstance(weights, MoeWeights) else make_weights(weights)
     T = h.shape[0]
+    _shape(h, "h", (T, cfg.d), (torch.bfloat16,))
+    _shape(norm_g, "norm_g", (cfg.d,), (torch.bfloat16,))
+    _shape(bias, "bias", (cfg.n_experts,), (torch.float32,))
+    _shape(y, "y", (T, cfg.d), (torch.bfloat16,))
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     ev, ro = _events(stage_events), _routing(routing_out)
     _check(lib().moe_forward_block(ctypes.byref(cfg), ctypes.byref(mw), _p(norm_g), float(eps), _p(h), _p(bias), T,
@@ -314,6 +349,17 @@ def moe_dense_ffn(w_gate, w_up, w_down, x, y, s_gate=None, s_up=None, s_down=Non
     hidden, d = w_gate.shape
     wdt = MOE_E4M3 if w_gate.dtype == torch.uint8 else MOE_BF16
     T = x.shape[0]
+    wt = (torch.uint8,) if wdt == MOE_E4M3 else (torch.bfloat16,)
+    _shape(w_up, "w_up", (hidden, d), wt)
+    _shape(w_down, "w_down", (d, hidden), wt)
+    _shape(x, "x", (T, d), (torch.bfloat16,) if wdt == MOE_E4M3 else (torch.bfloat16, torch.float32))
+    _shape(y, "y", (T, d), _OUT)
+    if wdt == MOE_E4M3:
+        for n, t, shp in (("s_gate", s_gate, (hidden // 128, d // 128)), ("s_up", s_up, (hidden // 128, d // 128)),
+                          ("s_down", s_down, (d // 128, hidden // 128))):
+            if t is None:
+                raise ValueError(f"{n}: e4m3 weights need their block scales")
+            _shape(t, n, shp, (torch.float32,))
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     ev = _events(stage_events)
     _check(lib().moe_dense_ffn(d, hidden, _dtype_code(x), wdt, _p(w_gate), _p(w_up), _p(w_down), _p(s_gate),
