@@ -140,6 +140,20 @@ def test_prefill_sampled():
     assert_close_bf16(yb[torch.from_numpy(toks).long().to(DEV)], ref, REL)
 
 
+def test_large_batch_sampled():
+    """T = 65536, four times the skewed workload's batch: the multi-CTA permutation over
+    256 blocks, 589,824 permuted rows, several token chunks for every expert; routing
+    and permutation checked for all tokens, outputs on a sample."""
+    wl = WORKLOADS["prefill"]
+    W = inputs("prefill", "cuda")
+    T = 65536
+    x = make_x(wl, "cuda", T=T)
+    toks = _sample(T, 3, seed=3)
+    ref = oracle_y(wl, W, x, toks)
+    yb = run_forward(wl, W, x, torch.bfloat16)
+    assert_close_bf16(yb[torch.from_numpy(toks).long().to(DEV)], ref, REL)
+
+
 def test_skewed_sampled():
     wl = WORKLOADS["skewed"]
     W = inputs("skewed", "cuda")
