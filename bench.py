@@ -35,11 +35,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the kernel sources hash to the recorded value.  profile_decode is captured
 # directly (the gate/up GEMM streams 30 routed + 1 shared expert weight sets);
 # decode is that capture scaled by weight sets streamed, 146 / 31 (traffic grows
-# with the touched experts: the profile_decode capture reads 0.99994 x its
+# with the touched experts: the profile_decode capture moves 0.99998 x its
 # algorithmic bytes).
 NCU_TRAFFIC = {
-    "profile_decode": (1_822_874_368, "88be10ddbf705e57"),
-    "decode": (8_585_150_262, "88be10ddbf705e57"),
+    "profile_decode": (1_822_942_464, "b448e5aeed8f3701"),
+    "decode": (8_585_470_959, "b448e5aeed8f3701"),
 }
 
 
