@@ -52,6 +52,18 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The slowest rank's figure: every rank of the process group takes part (a no-op in
+    a single process).  Timings are device-measured per rank, then reduced here."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -410,10 +422,7 @@ def run_ours(args, wl):
     ms = t_start.elapsed_time(t_end) if flush is None else sum(e[0].elapsed_time(e[5]) for e in evs)
     stage_ms = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
                 for i, name in enumerate(moe.STAGES)}
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, dev)
     if moe.device_error() != 0:
         raise RuntimeError("device error word set during the timed steps")
 
@@ -440,10 +449,7 @@ def run_ours(args, wl):
         e2e_step()
         e2e_evs[i][1].record(stream)
     torch.cuda.synchronize()
-    te = torch.tensor([sum(a.elapsed_time(b) for a, b in e2e_evs)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_evs), dev)
 
     # routed experts actually touched (for the byte accounting), through the ABI
     logits = torch.empty((T, wl.n_experts), dtype=torch.float32, device=dev)
@@ -580,10 +586,7 @@ def run_dense(args, wl):
     per_step = 4 + (2 if wl.fp8 else 1)  # tables, gather (+ quantisation), two GEMMs, cast
     if launches != per_step * args.steps or moe.device_error() != 0:
         raise RuntimeError(f"dense FFN: {launches} launches, device error word set or not as planned")
-    tt = torch.tensor([t0.elapsed_time(t1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-    ms = float(tt.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), dev)
     stage_ms = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, name in enumerate(moe.STAGES)}
     # end to end with host buffers
     x_host, y_host = x.cpu().pin_memory(), torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
@@ -596,9 +599,8 @@ def run_dense(args, wl):
         y_host.copy_(y, non_blocking=True)
         e_evs[i][1].record(stream)
     torch.cuda.synchronize()
-    te = torch.tensor([sum(a.elapsed_time(b) for a, b in e_evs)], dtype=torch.float64, device=dev)
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_evs), dev)
     if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
@@ -631,7 +633,7 @@ def run_dense(args, wl):
                    "T": T, "l2": f"inputs larger than L2: {3 * d * Hd * wb / 1e9:.2f} GB of weights stream every step",
                    "parallelism": f"replicas x{world} (no data-path collective)"},
         "roofline": kr, "layer_roofline": lr, "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
-        "e2e": {"value": round(world * T * args.steps / (float(te.item()) / 1e3), 1), "unit": UNIT,
+        "e2e": {"value": round(world * T * args.steps / (e2e_ms / 1e3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": x.numel() * x.element_size(), "d2h_bytes_per_step": y.numel() * y.element_size()},
         "gpu_launches": launches, "clocks": clk.summary(), "kernel_source": kernel_source_hash(),
     }
