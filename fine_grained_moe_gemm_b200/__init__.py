@@ -21,6 +21,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+_DEFAULT_LIB_PATH = LIB_PATH
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "moe.h")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_DEVICE, MOE_ERR_CUDA = range(6)
@@ -56,10 +57,19 @@ class MoeWeights(ctypes.Structure):
 
 
 def lib():
-    """The loaded ``libmoe_b200.so``; raises if it has not been built."""
+    """The loaded ``libmoe_b200.so``.  The in-tree library is (re)built first when it is
+    missing or older than its sources and nvcc is at hand; without it the call raises
+    (there is no CPU fallback)."""
     global _lib
     with _lock:
         if _lib is None:
+            if os.path.abspath(LIB_PATH) == os.path.abspath(_DEFAULT_LIB_PATH):
+                try:
+                    from . import build as _build
+                    _build.build()  # a no-op when the library is newer than every source
+                except Exception as e:
+                    if not os.path.exists(LIB_PATH):
+                        raise RuntimeError(f"{LIB_PATH} is missing and could not be built: {e}") from e
             if not os.path.exists(LIB_PATH):
                 raise RuntimeError(f"{LIB_PATH} is missing: build it with fine_grained_moe_gemm_b200.build.build() "
                                    "(there is no CPU fallback)")
