@@ -569,13 +569,16 @@ moe_status run_experts(const moe_config* cfg, const moe_weights* wt, const Works
     auto mark = [&](int i) {
         if (events && events->ev[i]) cudaEventRecord((cudaEvent_t)events->ev[i], s);
     };
+    // one group of all T rows in token order (the dense FFN) with bf16 x: the token
+    // operand is x itself, no gathered copy
+    const bool direct_b = E == 0 && !fp8 && cfg->act_dtype == MOE_BF16;
     if (fp8) {
         if ((!act_quantised && launch_quant_act(static_cast<const __nv_bfloat16*>(x), T, d, W.x_q, W.sx, s) != cudaSuccess) ||
             launch_gather_fp8(W.x_q, W.sx, d, W.row_tok, W.row_off + NG, rows_max, W.xq_perm, W.sxT, di.sm_count,
                               s) != cudaSuccess)
             return MOE_ERR_CUDA;
-    } else if (launch_gather(x, cfg->act_dtype == MOE_F32, d, W.row_tok, W.row_off + NG, rows_max, W.x_perm,
-                             di.sm_count, s) != cudaSuccess) {
+    } else if (!direct_b && launch_gather(x, cfg->act_dtype == MOE_F32, d, W.row_tok, W.row_off + NG, rows_max,
+                                          W.x_perm, di.sm_count, s) != cudaSuccess) {
         return MOE_ERR_CUDA;
     }
     mark(2);
@@ -601,7 +604,8 @@ moe_status run_experts(const moe_config* cfg, const moe_weights* wt, const Works
         g.s0 = g.a0;
         g.s1 = g.a1;
     }
-    if (!(fp8 ? map_u8(&g.b, W.xq_perm, rows_max, d, box_rows) : map_bf16(&g.b, W.x_perm, rows_max, d, box_rows)))
+    if (!(fp8 ? map_u8(&g.b, W.xq_perm, rows_max, d, box_rows)
+              : map_bf16(&g.b, direct_b ? x : W.x_perm, rows_max, d, box_rows)))
         return MOE_ERR_CUDA;
     g.item_off = W.item_gu;
     g.row_off = W.row_off;
