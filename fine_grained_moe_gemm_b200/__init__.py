@@ -157,6 +157,9 @@ def _dtype_code(t: torch.Tensor) -> int:
 def _dev(t: torch.Tensor, name: str):
     if t is not None and (not t.is_cuda or not t.is_contiguous()):
         raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if t is not None and t.device.index != torch.cuda.current_device():
+        # the library launches on the current device: a pointer into another GPU is not its memory
+        raise ValueError(f"{name} is on {t.device}, the current device is cuda:{torch.cuda.current_device()}")
 
 
 def _shape(t, name, shape, dtypes):

@@ -685,14 +685,14 @@ size_t gemm_args_size() { return sizeof(GemmArgs); }
 template <int MODE, int BN>
 static cudaError_t launch_gemm_t(const GemmArgs* args, int grid, cudaStream_t s) {
     using C = GemmCfg<MODE, BN>;
-    static bool attr_set[64] = {};
+    static std::atomic<bool> attr_set[64];  // once per device (a repeated set is harmless)
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && !attr_set[dev]) {
+    if (dev < 64 && !attr_set[dev].load(std::memory_order_relaxed)) {
         cudaError_t e = cudaFuncSetAttribute(moe_gemm_kernel<MODE, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
+        attr_set[dev].store(true, std::memory_order_relaxed);
     }
     note_launch();
     moe_gemm_kernel<MODE, BN><<<grid, GEMM_THREADS, C::SMEM_BYTES, s>>>(*args);
@@ -736,14 +736,14 @@ cudaError_t launch_gemm(int mode, int bn, const GemmArgs* args, int grid, cudaSt
 template <int MODE, int BN>
 static cudaError_t launch_gemm_fp8_t(const GemmArgs* args, int grid, cudaStream_t s) {
     using C = Fp8Cfg<MODE, BN>;
-    static bool attr_set[64] = {};
+    static std::atomic<bool> attr_set[64];  // once per device (a repeated set is harmless)
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && !attr_set[dev]) {
+    if (dev < 64 && !attr_set[dev].load(std::memory_order_relaxed)) {
         cudaError_t e = cudaFuncSetAttribute(moe_gemm_fp8_kernel<MODE, BN>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
+        attr_set[dev].store(true, std::memory_order_relaxed);
     }
     note_launch();
     moe_gemm_fp8_kernel<MODE, BN><<<grid, GEMM_THREADS, C::SMEM_BYTES, s>>>(*args);
@@ -774,14 +774,14 @@ cudaError_t launch_gemm_fp8(int mode, int bn, const GemmArgs* args, int grid, cu
 
 template <int MODE>
 static cudaError_t launch_gemm2_t(const GemmArgs* args, int grid, cudaStream_t s) {
-    static bool attr_set[64] = {};
+    static std::atomic<bool> attr_set[64];  // once per device (a repeated set is harmless)
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && !attr_set[dev]) {
+    if (dev < 64 && !attr_set[dev].load(std::memory_order_relaxed)) {
         cudaError_t e = cudaFuncSetAttribute(moe_gemm2_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              Gemm2Cfg::SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
+        attr_set[dev].store(true, std::memory_order_relaxed);
     }
     note_launch();
     moe_gemm2_kernel<MODE><<<grid, PAIR_THREADS, Gemm2Cfg::SMEM_BYTES, s>>>(*args);
@@ -798,14 +798,14 @@ cudaError_t launch_gemm2(int mode, const GemmArgs* args, int grid, cudaStream_t 
 
 template <int MODE>
 static cudaError_t launch_gemm2_fp8_t(const GemmArgs* args, int grid, cudaStream_t s) {
-    static bool attr_set[64] = {};
+    static std::atomic<bool> attr_set[64];  // once per device (a repeated set is harmless)
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && !attr_set[dev]) {
+    if (dev < 64 && !attr_set[dev].load(std::memory_order_relaxed)) {
         cudaError_t e = cudaFuncSetAttribute(moe_gemm2_fp8_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              Gemm2Fp8Cfg::SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
+        attr_set[dev].store(true, std::memory_order_relaxed);
     }
     note_launch();
     moe_gemm2_fp8_kernel<MODE><<<grid, GEMM_THREADS, Gemm2Fp8Cfg::SMEM_BYTES, s>>>(*args);
@@ -849,14 +849,14 @@ cudaError_t launch_select(const float* logits, const float* bias, int T, int E, 
                           float* w, cudaStream_t s, const float* parts, int n_parts) {
     const int blocks = (T + SELECT_WARPS - 1) / SELECT_WARPS;
     const size_t smem = (size_t)SELECT_WARPS * 2 * E * sizeof(float);
-    static bool attr_set[64] = {};
+    static std::atomic<bool> attr_set[64];  // once per device (a repeated set is harmless)
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && !attr_set[dev]) {
+    if (dev < 64 && !attr_set[dev].load(std::memory_order_relaxed)) {
         cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              SELECT_WARPS * 2 * 1024 * (int)sizeof(float));
         if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
+        attr_set[dev].store(true, std::memory_order_relaxed);
     }
     note_launch();
     select_kernel<<<blocks, SELECT_WARPS * 32, smem, s>>>(logits, bias, T, E, G, tg, k, idx, w,
@@ -868,13 +868,13 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s) {
     int WR = 8192 / a.E;
     WR = WR > 32 ? 32 : (WR < 1 ? 1 : WR);
     const size_t smem = (size_t)(PERM_SCAN_CAP + a.E + 64) * 4 + (size_t)2 * WR * a.E * 4;
-    static bool attr_set[64] = {};
+    static std::atomic<bool> attr_set[64];  // once per device (a repeated set is harmless)
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && !attr_set[dev]) {
+    if (dev < 64 && !attr_set[dev].load(std::memory_order_relaxed)) {
         cudaError_t e = cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
         if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
+        attr_set[dev].store(true, std::memory_order_relaxed);
     }
     note_launch();
     permute_kernel<<<1, PERM_THREADS, smem, s>>>(a, WR);
@@ -886,16 +886,16 @@ int permute_blocks(int T) { return (T + PERM_TB - 1) / PERM_TB; }
 cudaError_t launch_permute_multi(const PermuteArgs& a, int32_t* hist, cudaStream_t s) {
     const int nb = permute_blocks(a.T);
     const size_t smem_c = (size_t)(PERM_TB / 32) * a.E * 4;
-    static bool attr_set[64] = {};
+    static std::atomic<bool> attr_set[64];  // once per device (a repeated set is harmless)
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && !attr_set[dev]) {
+    if (dev < 64 && !attr_set[dev].load(std::memory_order_relaxed)) {
         cudaError_t e = cudaFuncSetAttribute(permute_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              64 * 1024);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
         if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
+        attr_set[dev].store(true, std::memory_order_relaxed);
     }
     note_launch();
     permute_count_kernel<<<nb, PERM_TB, smem_c, s>>>(a, hist);
