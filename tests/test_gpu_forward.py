@@ -130,6 +130,21 @@ def test_decode(T):
     assert_close_bf16(yb[torch.from_numpy(toks).long().to(DEV)], ref, REL)
 
 
+@pytest.mark.parametrize("T", [1000, 2048])
+def test_mid_batches_sampled(T):
+    """The single-CTA kernels' wider token tiles at full size: ~31 rows per expert
+    (64-row tiles) at T = 1000 and ~64 (128-row tiles) at T = 2048."""
+    wl = WORKLOADS["prefill"]
+    W = inputs("prefill", "cuda")
+    x = make_x(wl, "cuda", T=T)
+    toks = _sample(T, 4, seed=T)
+    ref = oracle_y(wl, W, x, toks)
+    yb = run_forward(wl, W, x, torch.bfloat16)
+    assert_close_bf16(yb[torch.from_numpy(toks).long().to(DEV)], ref, REL)
+    cfg = cfg_of(wl)
+    assert moe.forward_plan(cfg, T)["token_tile"] == (64 if T == 1000 else 128)
+
+
 def test_prefill_sampled():
     wl = WORKLOADS["prefill"]
     W = inputs("prefill", "cuda")

@@ -102,7 +102,7 @@ def test_fp8_tiny_full(T):
     assert_close_bf16(run(wl, W, x, torch.bfloat16), ref, REL)
 
 
-@pytest.mark.parametrize("T", [8192, 1, 37, 300])
+@pytest.mark.parametrize("T", [8192, 1, 37, 300, 1000, 4096])
 def test_fp8_deepseek_sampled(T):
     wl, W = fp8_inputs("fp8")
     x = W["x"] if T == wl.T else make_x(wl, DEV, T=T)
