@@ -82,38 +82,54 @@ __device__ __forceinline__ void warp_best(float& v, int& id) {
     }
 }
 
-constexpr int SELECT_WARPS = 8;
+constexpr int SELECT_THREADS = 256;
+constexpr int MAX_ROUTER_SPLITS = 16;
 
-__global__ void __launch_bounds__(SELECT_WARPS * 32) select_kernel(const float* logits,
-                                                                   const float* __restrict__ bias, int T, int E,
-                                                                   int G, int topk_groups, int k,
-                                                                   int32_t* __restrict__ idx_out,
-                                                                   float* __restrict__ w_out,
-                                                                   const float* __restrict__ parts, int n_parts) {
+// tpb tokens per CTA (1 at small T, where latency rules, else up to 8): all
+// threads sum the router's K-split partials (each expert's in split order) and
+// apply sigmoid and bias into shared memory; then warp w takes the decisions
+// of token w.
+__global__ void __launch_bounds__(SELECT_THREADS) select_kernel(float* __restrict__ logits,
+                                                                const float* __restrict__ bias, int T, int E,
+                                                                int G, int topk_groups, int k,
+                                                                int32_t* __restrict__ idx_out,
+                                                                float* __restrict__ w_out,
+                                                                const float* __restrict__ parts, int n_parts,
+                                                                int tpb) {
     extern __shared__ float ssm[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = blockIdx.x * SELECT_WARPS + warp;
-    if (t >= T) return;  // uniform per warp
-    float* s = ssm + (size_t)warp * 2 * E;
-    float* b = s + E;
-    const float* l = logits + (size_t)t * E;
-    for (int e = lane; e < E; e += 32) {
+    const int t0 = blockIdx.x * tpb;
+    for (int i = threadIdx.x; i < tpb * E; i += SELECT_THREADS) {
+        const int tl = i / E, e = i - tl * E;
+        const int t = t0 + tl;
+        if (t >= T) break;  // i only grows
+        float* l = logits + (size_t)t * E;
         float lv;
         if (parts) {
             // split-K router: the partial logits summed in split order, stored as the logits
-            lv = parts[(size_t)t * E + e];
-            for (int p = 1; p < n_parts; ++p) lv = __fadd_rn(lv, parts[((size_t)p * T + t) * E + e]);
-            const_cast<float*>(l)[e] = lv;
+            float pv[MAX_ROUTER_SPLITS];
+#pragma unroll
+            for (int p = 0; p < MAX_ROUTER_SPLITS; ++p)
+                pv[p] = p < n_parts ? parts[((size_t)p * T + t) * E + e] : 0.0f;
+            lv = pv[0];
+#pragma unroll
+            for (int p = 1; p < MAX_ROUTER_SPLITS; ++p)
+                if (p < n_parts) lv = __fadd_rn(lv, pv[p]);
+            l[e] = lv;
         } else {
             lv = l[e];
         }
         float sv = sigmoid_spec(lv);
         float bv = __fadd_rn(sv, bias[e]);
         if (bv == 0.0f) bv = 0.0f;
-        s[e] = sv;
-        b[e] = bv;
+        ssm[(size_t)tl * 2 * E + e] = sv;
+        ssm[(size_t)tl * 2 * E + E + e] = bv;
     }
-    __syncwarp();
+    __syncthreads();
+    const int t = t0 + warp;
+    if (warp >= tpb || t >= T) return;  // uniform per warp
+    float* s = ssm + (size_t)warp * 2 * E;
+    float* b = s + E;
     const int gs = E / G;
     // group scores (lane g owns group g)
     float gsc = -INFINITY;
@@ -847,20 +863,25 @@ cudaError_t launch_router_f32(const float* x, const __nv_bfloat16* wr, int T, in
 
 cudaError_t launch_select(const float* logits, const float* bias, int T, int E, int G, int tg, int k, int32_t* idx,
                           float* w, cudaStream_t s, const float* parts, int n_parts) {
-    const int blocks = (T + SELECT_WARPS - 1) / SELECT_WARPS;
-    const size_t smem = (size_t)SELECT_WARPS * 2 * E * sizeof(float);
+    if (n_parts > MAX_ROUTER_SPLITS) return cudaErrorInvalidValue;
+    // few tokens: one per CTA (the partial sums and the decisions spread over
+    // more SMs); many: eight per CTA (eight deciding warps a CTA)
+    const int tpb = T >= 8 * 148 ? SELECT_THREADS / 32 : 1;
+    const size_t smem = (size_t)tpb * 2 * E * sizeof(float);  // <= 64 KB (E <= 1024)
     static std::atomic<bool> attr_set[64];  // once per device (a repeated set is harmless)
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_set[dev].load(std::memory_order_relaxed)) {
         cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             SELECT_WARPS * 2 * 1024 * (int)sizeof(float));
+                                             (SELECT_THREADS / 32) * 2 * 1024 * (int)sizeof(float));
         if (e != cudaSuccess) return e;
         attr_set[dev].store(true, std::memory_order_relaxed);
     }
     note_launch();
-    select_kernel<<<blocks, SELECT_WARPS * 32, smem, s>>>(logits, bias, T, E, G, tg, k, idx, w,
-                                                         n_parts > 1 ? parts : nullptr, n_parts);
+    // logits is written only when the partials are summed here (split-K router)
+    select_kernel<<<(T + tpb - 1) / tpb, SELECT_THREADS, smem, s>>>(const_cast<float*>(logits), bias, T, E, G, tg,
+                                                                    k, idx, w, n_parts > 1 ? parts : nullptr,
+                                                                    n_parts, tpb);
     return cudaGetLastError();
 }
 
