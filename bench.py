@@ -52,6 +52,59 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
+def time_e2e(e2e_step, steps: int, warmup: int, streams, device, barrier=lambda: None, flush=None):
+    """End-to-end step times with host buffers, in ms over `steps` steps: (serial, pipelined).
+    e2e_step(i, s) enqueues step i (copy in, layer, copy out) on stream s, alternating between
+    two buffer sets by i % 2.  serial: one stream, per-step events summed (an L2 flush between
+    steps when `flush` is given).  pipelined: steps alternate between the two streams, so one
+    step's copies overlap the other's kernels; first copy to last copy.  None without a flush
+    only (small inputs are measured serially)."""
+    import torch
+
+    def pipelined(n):
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(streams[0])
+        streams[1].wait_event(t0)
+        for i in range(n):
+            e2e_step(i, streams[i % 2])
+        done = torch.cuda.Event()
+        done.record(streams[1])
+        streams[0].wait_event(done)
+        t1.record(streams[0])
+        return t0, t1
+
+    for i in range(max(warmup, 1)):
+        e2e_step(i, streams[0])
+    pipelined(2 * max(warmup, 1))
+    torch.cuda.synchronize()
+    barrier()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        if flush is not None:
+            flush.fill_(i & 0xff)
+        evs[i][0].record(streams[0])
+        e2e_step(i, streams[0])
+        evs[i][1].record(streams[0])
+    torch.cuda.synchronize()
+    serial = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), device)
+    pipe = None
+    if flush is None:
+        barrier()
+        p0, p1 = pipelined(steps)
+        torch.cuda.synchronize()
+        pipe = max_over_ranks(p0.elapsed_time(p1), device)
+    return serial, pipe
+
+
+def e2e_entry(tokens: float, serial_ms: float, pipe_ms, h2d: int, d2h: int, api: str) -> dict:
+    best = pipe_ms if pipe_ms is not None else serial_ms
+    return {"value": round(tokens / (best / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "api": api, "mode": "pipelined" if pipe_ms is not None else "serial",
+            "serial_value": round(tokens / (serial_ms / 1e3), 1),
+            "pipeline": ("steps alternate between two streams and two buffer sets: one step's host copies "
+                         "overlap the other step's kernels") if pipe_ms is not None else None}
+
+
 def max_over_ranks(x: float, device) -> float:
     """The slowest rank's figure: every rank of the process group takes part (a no-op in
     a single process).  Timings are device-measured per rank, then reduced here."""
@@ -426,30 +479,39 @@ def run_ours(args, wl):
     if moe.device_error() != 0:
         raise RuntimeError("device error word set during the timed steps")
 
-    # end to end through the public API with host buffers: pinned x in, y out
-    x_host = x.cpu().pin_memory()
-    y_host = torch.empty((T, wl.d), dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty_like(x)
+    # end to end with host buffers: pinned x in, y out, every step.  The layer goes through
+    # moe_forward_host (the C ABI call that takes host buffers and does the copies); the block,
+    # which has no host entry point, copies around moe_forward_block.  Measured two ways:
+    #   serial     one stream: copy in, layer, copy out, step after step (per-step events, summed)
+    #   pipelined  steps alternate between two streams with two workspaces, so the copies of
+    #              one step run on the copy engines while the other step's kernels run (the
+    #              loop a server runs); timed from the first copy to the last one.
     e2e_steps = max(1, args.steps)
+    x_host = x.cpu().pin_memory()
+    y_hosts = [torch.empty((T, wl.d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    streams = [stream, torch.cuda.Stream()]
+    if block:
+        x_devs = [torch.empty_like(x) for _ in range(2)]
+        y_devs = [y, torch.empty_like(y)]
+        e2e_ws = [ws, torch.empty_like(ws)]
+    else:
+        hws = moe.host_workspace_size(cfg, T, torch.bfloat16)
+        e2e_ws = [torch.empty(hws, dtype=torch.uint8, device=dev) for _ in range(2)]
 
-    def e2e_step():
-        x_dev.copy_(x_host, non_blocking=True)
-        forward(x_dev)
-        y_host.copy_(y, non_blocking=True)
+    def e2e_step(i, s):
+        j = i % 2
+        if block:
+            with torch.cuda.stream(s):
+                x_devs[j].copy_(x_host, non_blocking=True)
+                moe.moe_forward_block(cfg, weights, norm_g, x_devs[j], bias, y_devs[j], workspace=e2e_ws[j],
+                                      stream=s)
+                y_hosts[j].copy_(y_devs[j], non_blocking=True)
+        else:
+            moe.moe_forward_host(cfg, weights, x_host, bias, y_hosts[j], workspace=e2e_ws[j], stream=s)
 
-    for _ in range(max(args.warmup, 1)):
-        e2e_step()
-    torch.cuda.synchronize()
-    barrier()
-    e2e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
-    for i in range(e2e_steps):
-        if flush is not None:
-            flush.fill_(i & 0xff)
-        e2e_evs[i][0].record(stream)
-        e2e_step()
-        e2e_evs[i][1].record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_evs), dev)
+    e2e_serial_ms, e2e_pipe_ms = time_e2e(e2e_step, e2e_steps, args.warmup, streams, dev, barrier, flush)
+    if moe.device_error() != 0:
+        raise RuntimeError("device error word set during the end-to-end steps")
 
     # routed experts actually touched (for the byte accounting), through the ABI
     logits = torch.empty((T, wl.n_experts), dtype=torch.float32, device=dev)
@@ -511,9 +573,9 @@ def run_ours(args, wl):
             "roofline": kr,
             "layer_roofline": lr,
             "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
-            "e2e": {"value": round(world * T * e2e_steps / (e2e_ms / 1e3), 1), "unit": UNIT,
-                    "h2d_bytes_per_step": x.numel() * x.element_size(),
-                    "d2h_bytes_per_step": y.numel() * y.element_size()},
+            "e2e": e2e_entry(world * T * e2e_steps, e2e_serial_ms, e2e_pipe_ms, x.numel() * x.element_size(),
+                             y.numel() * y.element_size(),
+                             "moe_forward_block + copies" if block else "moe_forward_host (host buffers)"),
             "gpu_launches": launches,
             "plan": plan,
             "clocks": clk.summary(),
@@ -607,18 +669,24 @@ def run_dense(args, wl):
         raise RuntimeError(f"dense FFN: {launches} launches, device error word set or not as planned")
     ms = max_over_ranks(t0.elapsed_time(t1), dev)
     stage_ms = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, name in enumerate(moe.STAGES)}
-    # end to end with host buffers
-    x_host, y_host = x.cpu().pin_memory(), torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty_like(x)
-    e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for i in range(args.steps):
-        e_evs[i][0].record(stream)
-        x_dev.copy_(x_host, non_blocking=True)
-        forward(x_dev)
-        y_host.copy_(y, non_blocking=True)
-        e_evs[i][1].record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_evs), dev)
+    # end to end with host buffers (copies around moe_dense_ffn), serial and pipelined as for the layer
+    x_host = x.cpu().pin_memory()
+    y_hosts = [torch.empty((T, d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    x_devs, y_devs, wss = [torch.empty_like(x) for _ in range(2)], [y, torch.empty_like(y)], [ws, torch.empty_like(ws)]
+
+    def e2e_step(i, s):
+        j = i % 2
+        with torch.cuda.stream(s):
+            x_devs[j].copy_(x_host, non_blocking=True)
+            moe.moe_dense_ffn(W["w_gate"], W["w_up"], W["w_down"], x_devs[j], y_devs[j], W.get("s_gate"),
+                              W.get("s_up"), W.get("s_down"), workspace=wss[j], stream=s)
+            y_hosts[j].copy_(y_devs[j], non_blocking=True)
+
+    barrier = (lambda: dist.barrier()) if world > 1 else (lambda: None)
+    e2e_serial_ms, e2e_pipe_ms = time_e2e(e2e_step, args.steps, args.warmup, [stream, torch.cuda.Stream()], dev,
+                                          barrier)
+    if moe.device_error() != 0:
+        raise RuntimeError("dense FFN: device error word set during the end-to-end steps")
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -652,8 +720,8 @@ def run_dense(args, wl):
                    "T": T, "l2": f"inputs larger than L2: {3 * d * Hd * wb / 1e9:.2f} GB of weights stream every step",
                    "parallelism": f"replicas x{world} (no data-path collective)"},
         "roofline": kr, "layer_roofline": lr, "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
-        "e2e": {"value": round(world * T * args.steps / (e2e_ms / 1e3), 1), "unit": UNIT,
-                "h2d_bytes_per_step": x.numel() * x.element_size(), "d2h_bytes_per_step": y.numel() * y.element_size()},
+        "e2e": e2e_entry(world * T * args.steps, e2e_serial_ms, e2e_pipe_ms, x.numel() * x.element_size(),
+                         y.numel() * y.element_size(), "moe_dense_ffn + copies"),
         "gpu_launches": launches, "clocks": clk.summary(), "kernel_source": kernel_source_hash(),
     }
     line["config"]["launch"] = "CUDA-graph replay of the captured step" if graph is not None else "eager"

@@ -87,6 +87,11 @@ def lib():
             L.moe_forward_ex.restype = I
             L.moe_forward_ex.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, I, P, I, I, P,
                                          ctypes.c_size_t, P, P, P]
+            L.moe_host_workspace_size.restype = ctypes.c_size_t
+            L.moe_host_workspace_size.argtypes = [ctypes.POINTER(MoeConfig), I, I]
+            L.moe_forward_host.restype = I
+            L.moe_forward_host.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, I, P, I, I, P,
+                                           ctypes.c_size_t, P]
             L.moe_rmsnorm.restype = I
             L.moe_rmsnorm.argtypes = [P, P, ctypes.c_float, I, I, P, P, P, P]
             L.moe_block_workspace_size.restype = ctypes.c_size_t
@@ -290,6 +295,38 @@ def moe_forward(cfg: MoeConfig, weights, x, bias, y, accumulate: bool = False, w
                                 1 if accumulate else 0, _p(workspace), ws_bytes, _stream(stream),
                                 ctypes.byref(ev) if ev is not None else None,
                                 ctypes.byref(ro) if ro is not None else None), "moe_forward")
+
+
+def host_workspace_size(cfg: MoeConfig, T: int, y_dtype=torch.bfloat16) -> int:
+    """Device workspace bytes of ``moe_forward_host`` for up to T tokens."""
+    code = MOE_F32 if y_dtype == torch.float32 else MOE_BF16
+    return int(lib().moe_host_workspace_size(ctypes.byref(cfg), int(T), code))
+
+
+def _host(t: torch.Tensor, name: str):
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous host (CPU) tensor")
+
+
+def moe_forward_host(cfg: MoeConfig, weights, x_host, bias, y_host, accumulate: bool = False, workspace=None,
+                     stream=None):
+    """y_host (+)= MoE(x_host) with the activations in host memory: the call enqueues the copy in, the layer and
+    the copy out on ``stream`` and returns; ``y_host`` holds the result once the stream has passed that work.
+    Pin both host tensors (``pin_memory()``) for the copies to be asynchronous.  ``workspace``: a uint8 CUDA
+    tensor of at least ``host_workspace_size(cfg, T, y_host.dtype)`` bytes."""
+    _host(x_host, "x_host")
+    _host(y_host, "y_host")
+    for n, t in (("bias", bias), ("workspace", workspace)):
+        _dev(t, n)
+    mw = weights if isinstance(weights, MoeWeights) else make_weights(weights)
+    T = x_host.shape[0]
+    _shape(x_host, "x_host", (T, cfg.d), _ACT.get(cfg.act_dtype, ()))
+    _shape(bias, "bias", (cfg.n_experts,), (torch.float32,))
+    _shape(y_host, "y_host", (T, cfg.d), _OUT)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().moe_forward_host(ctypes.byref(cfg), ctypes.byref(mw), _p(x_host), _p(bias), T, _p(y_host),
+                                  _dtype_code(y_host), 1 if accumulate else 0, _p(workspace), ws_bytes,
+                                  _stream(stream)), "moe_forward_host")
 
 
 def selftest_wait_timeout(limit_ns: int = 1_000_000, stream=None):

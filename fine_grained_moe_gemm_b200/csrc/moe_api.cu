@@ -292,6 +292,35 @@ moe_status route_impl(const moe_config* c, const DevInfo& di, const void* x, con
 
 size_t xhat_bytes(const moe_config* c, int T) { return ((size_t)T * c->d * 2 + 255) & ~(size_t)255; }
 
+// The checks moe_forward makes before it enqueues anything (T == 0 passes).
+moe_status check_forward_args(const moe_config* cfg, const moe_weights* wt, const void* x, const float* bias, int T,
+                              const void* y, moe_dtype y_dtype, int accumulate, const void* workspace,
+                              size_t ws_bytes) {
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (T < 0 || (y_dtype != MOE_F32 && y_dtype != MOE_BF16) || (accumulate != 0 && accumulate != 1))
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!wt || !x || !bias || !y || !workspace) return MOE_ERR_INVALID_ARG;
+    if (!wt->w_router || !wt->w_gate || !wt->w_up || !wt->w_down) return MOE_ERR_INVALID_ARG;
+    if (cfg->n_shared && (!wt->ws_gate || !wt->ws_up || !wt->ws_down)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(wt->w_router) || !aligned16(wt->w_gate) ||
+        !aligned16(wt->w_up) || !aligned16(wt->w_down) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->n_shared && (!aligned16(wt->ws_gate) || !aligned16(wt->ws_up) || !aligned16(wt->ws_down)))
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->weight_dtype == MOE_E4M3) {
+        if (cfg->act_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+        if (!wt->s_gate || !wt->s_up || !wt->s_down) return MOE_ERR_INVALID_ARG;
+        if (cfg->n_shared && (!wt->ss_gate || !wt->ss_up || !wt->ss_down)) return MOE_ERR_INVALID_ARG;
+    }
+    if (ws_bytes < layout(cfg, T, nullptr).bytes) return MOE_ERR_WORKSPACE;
+    return MOE_OK;
+}
+
+size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
+size_t dtype_bytes(moe_dtype t) { return t == MOE_F32 ? 4 : t == MOE_BF16 ? 2 : 1; }
+
 moe_status forward_impl(const moe_config* cfg, const moe_weights* wt, const void* x, const float* bias, int T,
                         void* y, moe_dtype y_dtype, int accumulate, void* workspace, size_t ws_bytes,
                         moe_stream_t stream, const moe_stage_events* events, const moe_routing_out* routing,
@@ -543,6 +572,41 @@ moe_status moe_forward_block(const moe_config* cfg, const moe_weights* wt, const
     return forward_impl(cfg, wt, h, bias, T, y, MOE_BF16, 0, workspace, ws_bytes, stream, events, routing, norm_g, eps);
 }
 
+size_t moe_host_workspace_size(const moe_config* cfg, int T_max, moe_dtype y_dtype) {
+    if (y_dtype != MOE_F32 && y_dtype != MOE_BF16) return 0;
+    const size_t base = moe_workspace_size(cfg, T_max);
+    if (!base) return 0;
+    const size_t n = (size_t)T_max * cfg->d;
+    return round256(base) + round256(n * dtype_bytes(cfg->act_dtype)) + round256(n * dtype_bytes(y_dtype));
+}
+
+moe_status moe_forward_host(const moe_config* cfg, const moe_weights* wt, const void* x_host, const float* bias,
+                            int T, void* y_host, moe_dtype y_dtype, int accumulate, void* workspace, size_t ws_bytes,
+                            moe_stream_t stream) {
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (T < 0 || (y_dtype != MOE_F32 && y_dtype != MOE_BF16)) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return check_forward_args(cfg, wt, x_host, bias, 0, y_host, y_dtype, accumulate, workspace, ws_bytes);
+    if (!x_host || !y_host || !workspace) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < moe_host_workspace_size(cfg, T, y_dtype)) return MOE_ERR_WORKSPACE;
+    // the device copies of x and y sit behind the layer's own workspace
+    const size_t fw = round256(moe_workspace_size(cfg, T));
+    const size_t xb = (size_t)T * cfg->d * dtype_bytes(cfg->act_dtype);
+    const size_t yb = (size_t)T * cfg->d * dtype_bytes(y_dtype);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    void* xd = ws + fw;
+    void* yd = ws + fw + round256(xb);
+    if ((st = check_forward_args(cfg, wt, xd, bias, T, yd, y_dtype, accumulate, ws, fw)) != MOE_OK) return st;
+    DevInfo di;
+    if ((st = check_device(&di)) != MOE_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(xd, x_host, xb, cudaMemcpyHostToDevice, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (accumulate && cudaMemcpyAsync(yd, y_host, yb, cudaMemcpyHostToDevice, s) != cudaSuccess) return MOE_ERR_CUDA;
+    st = forward_impl(cfg, wt, xd, bias, T, yd, y_dtype, accumulate, ws, fw, stream, nullptr, nullptr, nullptr, 0.0f);
+    if (st != MOE_OK) return st;
+    return cudaMemcpyAsync(y_host, yd, yb, cudaMemcpyDeviceToHost, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 }  // extern "C"
 
 namespace {
@@ -694,26 +758,9 @@ moe_status forward_impl(const moe_config* cfg, const moe_weights* wt, const void
                         void* y, moe_dtype y_dtype, int accumulate, void* workspace, size_t ws_bytes,
                         moe_stream_t stream, const moe_stage_events* events, const moe_routing_out* routing,
                         const void* norm_g, float eps) {
-    moe_status st = check_config(cfg);
-    if (st != MOE_OK) return st;
-    if (T < 0 || (y_dtype != MOE_F32 && y_dtype != MOE_BF16) || (accumulate != 0 && accumulate != 1))
-        return MOE_ERR_INVALID_ARG;
-    if (T == 0) return MOE_OK;
-    if (!wt || !x || !bias || !y || !workspace) return MOE_ERR_INVALID_ARG;
-    if (!wt->w_router || !wt->w_gate || !wt->w_up || !wt->w_down) return MOE_ERR_INVALID_ARG;
-    if (cfg->n_shared && (!wt->ws_gate || !wt->ws_up || !wt->ws_down)) return MOE_ERR_INVALID_ARG;
-    if (!aligned16(x) || !aligned16(y) || !aligned16(wt->w_router) || !aligned16(wt->w_gate) ||
-        !aligned16(wt->w_up) || !aligned16(wt->w_down) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
-        return MOE_ERR_INVALID_ARG;
-    if (cfg->n_shared && (!aligned16(wt->ws_gate) || !aligned16(wt->ws_up) || !aligned16(wt->ws_down)))
-        return MOE_ERR_INVALID_ARG;
+    moe_status st = check_forward_args(cfg, wt, x, bias, T, y, y_dtype, accumulate, workspace, ws_bytes);
+    if (st != MOE_OK || T == 0) return st;
     const bool fp8 = cfg->weight_dtype == MOE_E4M3;
-    if (fp8) {
-        if (cfg->act_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
-        if (!wt->s_gate || !wt->s_up || !wt->s_down) return MOE_ERR_INVALID_ARG;
-        if (cfg->n_shared && (!wt->ss_gate || !wt->ss_up || !wt->ss_down)) return MOE_ERR_INVALID_ARG;
-    }
-    if (ws_bytes < layout(cfg, T, nullptr).bytes) return MOE_ERR_WORKSPACE;
     DevInfo di;
     if ((st = check_device(&di)) != MOE_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;

@@ -244,6 +244,35 @@ MOE_API moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* w, c
                                   size_t ws_bytes, moe_stream_t stream, const moe_stage_events* events,
                                   const moe_routing_out* routing);
 
+/* Bytes of device workspace moe_forward_host needs for up to T_max tokens with
+ * output type y_dtype: moe_workspace_size(cfg, T_max) plus the device copies of
+ * x and y, each rounded up to 256 bytes (0 on invalid arguments). */
+MOE_API size_t moe_host_workspace_size(const moe_config* cfg, int T_max, moe_dtype y_dtype);
+
+/* moe_forward on host buffers: the layer as a host program calls it, with the
+ * activations in host memory and the weights, the bias and the workspace on
+ * the device.  This entry point has no counterpart on the pages; it is the
+ * copy in, the layer of moe_forward and the copy out in one call.
+ *   x_host [T, d] cfg->act_dtype and y_host [T, d] y_dtype are host memory.
+ *   The call enqueues on `stream`: the copy of x_host into the workspace, with
+ *   accumulate = 1 the copy of y_host in (the residual), moe_forward on the
+ *   device copies, and the copy of the result back into y_host.  It returns
+ *   without waiting: y_host holds the result once the stream has passed that
+ *   work (cudaStreamSynchronize, or an event recorded after the call), and
+ *   both host buffers must stay valid and untouched until then.
+ *   With page-locked host memory (cudaHostAlloc, cudaHostRegister) the copies
+ *   run on the copy engines while other streams compute, so two calls on two
+ *   streams with two workspaces overlap one call's copies with the other's
+ *   kernels.  With pageable memory the driver stages the copies and the call
+ *   may block the host until they are done.
+ *   workspace: device, 256-byte aligned, ws_bytes >= moe_host_workspace_size(
+ *   cfg, T, y_dtype); its tail holds the device copies of x and y.
+ * Every argument is checked before anything is enqueued; results and errors as
+ * moe_forward, MOE_ERR_CUDA when a copy cannot be enqueued. */
+MOE_API moe_status moe_forward_host(const moe_config* cfg, const moe_weights* w, const void* x_host,
+                                    const float* bias, int T, void* y_host, moe_dtype y_dtype, int accumulate,
+                                    void* workspace, size_t ws_bytes, moe_stream_t stream);
+
 /* Pre-norm ("DeepSeek-V3" llm-vis, "RMSNorm" box: every token vector is
  * rescaled to unit RMS over its features with eps = 1e-6, cast back to bf16,
  * then multiplied by the learned per-feature gain):

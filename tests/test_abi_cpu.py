@@ -148,3 +148,30 @@ def test_dense_arguments(L):
 def test_selftest_arguments(L):
     assert L.moe_selftest_wait_timeout(0, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_selftest_wait_timeout(2_000_000_000, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_host_entry_arguments(L):
+    """moe_forward_host: every argument is checked before anything is enqueued, so the
+    errors below come back without a device."""
+    cfg = cfg_of(WORKLOADS["decode"])
+    P = ctypes.c_void_p
+    for T in (1, 128, 4096):
+        for yd, yb in ((moe.MOE_BF16, 2), (moe.MOE_F32, 4)):
+            need = L.moe_host_workspace_size(ctypes.byref(cfg), T, yd)
+            base = (moe.workspace_size(cfg, T) + 255) // 256 * 256
+            assert need == base + (T * 7168 * 2 + 255) // 256 * 256 + (T * 7168 * yb + 255) // 256 * 256
+    assert L.moe_host_workspace_size(ctypes.byref(cfg), 4, moe.MOE_E4M3) == 0
+    w = moe.MoeWeights(w_router=16, w_gate=16, w_up=16, w_down=16, ws_gate=16, ws_up=16, ws_down=16)
+    host = lambda T, x, y, yd, acc, ws: L.moe_forward_host(ctypes.byref(cfg), ctypes.byref(w), x, P(16), T, y, yd,
+                                                           acc, P(1 << 20), ws, None)
+    assert host(4, P(16), P(16), moe.MOE_BF16, 0, 1024) == moe.MOE_ERR_WORKSPACE
+    assert host(4, None, P(16), moe.MOE_BF16, 0, 1 << 30) == moe.MOE_ERR_INVALID_ARG     # no x
+    assert host(4, P(16), None, moe.MOE_BF16, 0, 1 << 30) == moe.MOE_ERR_INVALID_ARG     # no y
+    assert host(4, P(16), P(16), moe.MOE_E4M3, 0, 1 << 30) == moe.MOE_ERR_INVALID_ARG    # output dtype
+    assert host(4, P(16), P(16), moe.MOE_BF16, 2, 1 << 30) == moe.MOE_ERR_INVALID_ARG    # accumulate flag
+    assert host(-1, P(16), P(16), moe.MOE_BF16, 0, 1 << 30) == moe.MOE_ERR_INVALID_ARG
+    assert host(0, None, None, moe.MOE_BF16, 0, 0) == moe.MOE_OK                         # T = 0: a no-op
+    # host buffers need no alignment (they are copy sources and targets only)
+    nodev = L.moe_forward_host(ctypes.byref(cfg), ctypes.byref(moe.MoeWeights()), P(17), P(16), 4, P(19),
+                               moe.MOE_BF16, 0, P(1 << 20), 1 << 30, None)
+    assert nodev == moe.MOE_ERR_INVALID_ARG                                              # no weights
