@@ -35,11 +35,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the kernel sources hash to the recorded value.  profile_decode is captured
 # directly (the gate/up GEMM streams 30 routed + 1 shared expert weight sets);
 # decode is that capture scaled by weight sets streamed, 146 / 31 (traffic grows
-# with the touched experts: the profile_decode capture moves 0.99998 x its
+# with the touched experts: the profile_decode capture moves 0.99995 x its
 # algorithmic bytes).
 NCU_TRAFFIC = {
-    "profile_decode": (1_822_952_960, "bae114ca5feefad5"),
-    "decode": (8_585_520_392, "bae114ca5feefad5"),
+    "profile_decode": (1_822_885_120, "7d5f411566a278e1"),
+    "decode": (8_585_200_888, "7d5f411566a278e1"),
 }
 
 

@@ -92,6 +92,17 @@ def lib():
             L.moe_forward_host.restype = I
             L.moe_forward_host.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, I, P, I, I, P,
                                            ctypes.c_size_t, P]
+            L.moe_ep_max_send_rows.restype = I
+            L.moe_ep_max_send_rows.argtypes = [ctypes.POINTER(MoeConfig), I, I]
+            L.moe_ep_dispatch.restype = I
+            L.moe_ep_dispatch.argtypes = [ctypes.POINTER(MoeConfig), I, P, P, P, I, P, P, P, P, P, P, P]
+            L.moe_experts_routed_workspace_size.restype = ctypes.c_size_t
+            L.moe_experts_routed_workspace_size.argtypes = [ctypes.POINTER(MoeConfig), I, I]
+            L.moe_experts_routed.restype = I
+            L.moe_experts_routed.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), I, I, P, I, P, P,
+                                             P, P, ctypes.c_size_t, P]
+            L.moe_ep_combine.restype = I
+            L.moe_ep_combine.argtypes = [I, I, I, P, P, P, P, P, P]
             L.moe_rmsnorm.restype = I
             L.moe_rmsnorm.argtypes = [P, P, ctypes.c_float, I, I, P, P, P, P]
             L.moe_block_workspace_size.restype = ctypes.c_size_t
@@ -327,6 +338,78 @@ def moe_forward_host(cfg: MoeConfig, weights, x_host, bias, y_host, accumulate: 
     _check(lib().moe_forward_host(ctypes.byref(cfg), ctypes.byref(mw), _p(x_host), _p(bias), T, _p(y_host),
                                   _dtype_code(y_host), 1 if accumulate else 0, _p(workspace), ws_bytes,
                                   _stream(stream)), "moe_forward_host")
+
+
+def ep_max_send_rows(cfg: MoeConfig, T: int, n_ranks: int) -> int:
+    """Rows the dispatch of T tokens over n_ranks ranks can produce: T * min(k, n_ranks)."""
+    return int(lib().moe_ep_max_send_rows(ctypes.byref(cfg), int(T), int(n_ranks)))
+
+
+def moe_ep_dispatch(cfg: MoeConfig, n_ranks: int, topk_idx, topk_w, x, send_counts, send_offsets, send_tok, send_x,
+                    send_idx, send_w, stream=None):
+    """Expert-parallel dispatch: the rows this rank sends to each of ``n_ranks`` ranks (contiguous expert blocks),
+    rank-major, each token once per rank.  Output arrays hold ``ep_max_send_rows(cfg, T, n_ranks)`` rows."""
+    T = x.shape[0]
+    rows = ep_max_send_rows(cfg, T, n_ranks)
+    for n, t in (("topk_idx", topk_idx), ("topk_w", topk_w), ("x", x), ("send_counts", send_counts),
+                 ("send_offsets", send_offsets), ("send_tok", send_tok), ("send_x", send_x),
+                 ("send_idx", send_idx), ("send_w", send_w)):
+        _dev(t, n)
+    k = cfg.top_k
+    _shape(topk_idx, "topk_idx", (T, k), (torch.int32,))
+    _shape(topk_w, "topk_w", (T, k), (torch.float32,))
+    _shape(x, "x", (T, cfg.d), _ACT.get(cfg.act_dtype, ()))
+    _shape(send_counts, "send_counts", (n_ranks,), (torch.int32,))
+    _shape(send_offsets, "send_offsets", (n_ranks + 1,), (torch.int32,))
+    for n, t, shp, dt in (("send_tok", send_tok, (rows,), torch.int32), ("send_x", send_x, (rows, cfg.d), torch.bfloat16),
+                          ("send_idx", send_idx, (rows, k), torch.int32), ("send_w", send_w, (rows, k), torch.float32)):
+        if t.shape[0] < rows or tuple(t.shape[1:]) != shp[1:] or t.dtype != dt:
+            raise ValueError(f"{n}: shape {tuple(t.shape)} {t.dtype}, expected at least {shp} {dt}")
+    _check(lib().moe_ep_dispatch(ctypes.byref(cfg), int(n_ranks), _p(topk_idx), _p(topk_w), _p(x), T,
+                                 _p(send_counts), _p(send_offsets), _p(send_tok), _p(send_x), _p(send_idx),
+                                 _p(send_w), _stream(stream)), "moe_ep_dispatch")
+
+
+def experts_routed_workspace_size(cfg: MoeConfig, n_local: int, n_rows: int) -> int:
+    return int(lib().moe_experts_routed_workspace_size(ctypes.byref(cfg), int(n_local), int(n_rows)))
+
+
+def moe_experts_routed(cfg: MoeConfig, local_weights, expert_lo: int, n_local: int, x_rows, topk_idx, topk_w, y_rows,
+                       workspace=None, stream=None):
+    """y_rows = routed_scale * sum of the experts of block [expert_lo, expert_lo + n_local) over the given rows'
+    slots (the receiving side of the dispatch).  ``local_weights``: dict with the block's w_gate / w_up [n_local,
+    H, d] and w_down [n_local, d, H] (e4m3: plus s_gate / s_up / s_down)."""
+    for n, t in (("x_rows", x_rows), ("topk_idx", topk_idx), ("topk_w", topk_w), ("y_rows", y_rows),
+                 ("workspace", workspace)):
+        _dev(t, n)
+    mw = local_weights if isinstance(local_weights, MoeWeights) else make_weights(local_weights)
+    n = x_rows.shape[0]
+    _shape(x_rows, "x_rows", (n, cfg.d), (torch.bfloat16,))
+    _shape(topk_idx, "topk_idx", (n, cfg.top_k), (torch.int32,))
+    _shape(topk_w, "topk_w", (n, cfg.top_k), (torch.float32,))
+    _shape(y_rows, "y_rows", (n, cfg.d), (torch.float32,))
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().moe_experts_routed(ctypes.byref(cfg), ctypes.byref(mw), int(expert_lo), int(n_local), _p(x_rows), n,
+                                    _p(topk_idx), _p(topk_w), _p(y_rows), _p(workspace), ws_bytes,
+                                    _stream(stream)), "moe_experts_routed")
+
+
+def moe_ep_combine(back_rows, send_tok, y_acc, y=None, residual=None, stream=None):
+    """y_acc[send_tok[i]] += back_rows[i] (the partial sums the ranks returned), then y = bf16(y_acc + residual)
+    when ``y`` is given."""
+    for n, t in (("back_rows", back_rows), ("send_tok", send_tok), ("y_acc", y_acc), ("y", y),
+                 ("residual", residual)):
+        _dev(t, n)
+    T, d = y_acc.shape
+    n = back_rows.shape[0]
+    _shape(back_rows, "back_rows", (n, d), (torch.float32,))
+    _shape(y_acc, "y_acc", (T, d), (torch.float32,))
+    if send_tok.shape[0] < n or send_tok.dtype != torch.int32:
+        raise ValueError(f"send_tok: {tuple(send_tok.shape)} {send_tok.dtype}, expected at least ({n},) int32")
+    _shape(y, "y", (T, d), (torch.bfloat16,))
+    _shape(residual, "residual", (T, d), (torch.bfloat16,))
+    _check(lib().moe_ep_combine(T, d, n, _p(back_rows), _p(send_tok), _p(y_acc), _p(y), _p(residual),
+                                _stream(stream)), "moe_ep_combine")
 
 
 def selftest_wait_timeout(limit_ns: int = 1_000_000, stream=None):

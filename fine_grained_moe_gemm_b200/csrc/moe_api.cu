@@ -319,6 +319,20 @@ moe_status check_forward_args(const moe_config* cfg, const moe_weights* wt, cons
 }
 
 size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+// The layer restricted to a block of n_local routed experts (expert parallelism):
+// no selection (the routing is given), no shared expert, bf16 rows.
+bool local_cfg(const moe_config* cfg, int n_local, moe_config* c) {
+    if (check_config(cfg) != MOE_OK || n_local < 1 || n_local > cfg->n_experts) return false;
+    *c = *cfg;
+    c->n_experts = n_local;
+    c->n_groups = 1;
+    c->topk_groups = 1;
+    c->n_shared = 0;
+    c->shared_hidden = cfg->hidden;
+    c->act_dtype = MOE_BF16;
+    return true;
+}
 size_t dtype_bytes(moe_dtype t) { return t == MOE_F32 ? 4 : t == MOE_BF16 ? 2 : 1; }
 
 moe_status forward_impl(const moe_config* cfg, const moe_weights* wt, const void* x, const float* bias, int T,
@@ -605,6 +619,105 @@ moe_status moe_forward_host(const moe_config* cfg, const moe_weights* wt, const 
     st = forward_impl(cfg, wt, xd, bias, T, yd, y_dtype, accumulate, ws, fw, stream, nullptr, nullptr, nullptr, 0.0f);
     if (st != MOE_OK) return st;
     return cudaMemcpyAsync(y_host, yd, yb, cudaMemcpyDeviceToHost, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_ep_max_send_rows(const moe_config* cfg, int T, int n_ranks) {
+    if (check_config(cfg) != MOE_OK || T < 0 || n_ranks < 1) return 0;
+    return T * (cfg->top_k < n_ranks ? cfg->top_k : n_ranks);
+}
+
+moe_status moe_ep_dispatch(const moe_config* cfg, int n_ranks, const int32_t* topk_idx, const float* topk_w,
+                           const void* x, int T, int32_t* send_counts, int32_t* send_offsets, int32_t* send_tok,
+                           void* send_x, int32_t* send_idx, float* send_w, moe_stream_t stream) {
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (T < 0 || n_ranks < 1 || n_ranks > 32 || cfg->n_experts % n_ranks != 0) return MOE_ERR_INVALID_ARG;
+    if (!send_counts || !send_offsets) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!topk_idx || !topk_w || !x || !send_tok || !send_x || !send_idx || !send_w || !aligned16(x) ||
+                  !aligned16(send_x)))
+        return MOE_ERR_INVALID_ARG;
+    DevInfo di;
+    if ((st = check_device(&di)) != MOE_OK) return st;
+    return cuda_status(launch_ep_dispatch(topk_idx, topk_w, T, cfg->top_k, cfg->n_experts, n_ranks, x,
+                                          cfg->act_dtype == MOE_F32, cfg->d, send_counts, send_offsets, send_tok,
+                                          static_cast<__nv_bfloat16*>(send_x), send_idx, send_w, di.sm_count,
+                                          (cudaStream_t)stream));
+}
+
+size_t moe_experts_routed_workspace_size(const moe_config* cfg, int n_local, int n_rows_max) {
+    moe_config c;
+    if (!local_cfg(cfg, n_local, &c) || n_rows_max < 0) return 0;
+    return layout(&c, n_rows_max, nullptr).bytes;
+}
+
+moe_status moe_experts_routed(const moe_config* cfg, const moe_weights* wl, int expert_lo, int n_local,
+                              const void* x_rows, int n_rows, const int32_t* topk_idx, const float* topk_w,
+                              float* y_rows, void* workspace, size_t ws_bytes, moe_stream_t stream) {
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    moe_config c;
+    if (!local_cfg(cfg, n_local, &c) || expert_lo < 0 || expert_lo > cfg->n_experts - n_local || n_rows < 0)
+        return MOE_ERR_INVALID_ARG;
+    if (n_rows == 0) return MOE_OK;
+    if (!wl || !x_rows || !topk_idx || !topk_w || !y_rows || !workspace) return MOE_ERR_INVALID_ARG;
+    if (!wl->w_gate || !wl->w_up || !wl->w_down || !aligned16(wl->w_gate) || !aligned16(wl->w_up) ||
+        !aligned16(wl->w_down) || !aligned16(x_rows) || !aligned16(y_rows) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return MOE_ERR_INVALID_ARG;
+    if (c.weight_dtype == MOE_E4M3 && (!wl->s_gate || !wl->s_up || !wl->s_down)) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < layout(&c, n_rows, nullptr).bytes) return MOE_ERR_WORKSPACE;
+    DevInfo di;
+    if ((st = check_device(&di)) != MOE_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    const Workspace W = layout(&c, n_rows, workspace);
+    const Plan plan = make_plan(&c, n_rows, di.sm_count);
+    const int H = c.hidden, d = c.d;
+    // the permutation of the rows' slots of this block (other blocks' slots skipped) and the tile schedules
+    PermuteArgs pa;
+    memset(&pa, 0, sizeof(pa));
+    pa.idx = topk_idx;
+    pa.T = n_rows;
+    pa.k = c.top_k;
+    pa.E = n_local;
+    pa.id_lo = expert_lo;
+    pa.foreign_ok = 1;
+    pa.counts = W.counts;
+    pa.offsets = W.offsets;
+    pa.src = W.src;
+    pa.inv = W.inv;
+    pa.topk_w = topk_w;
+    pa.routed_scale = c.routed_scale;
+    pa.n_shared = 0;
+    pa.row_tok = W.row_tok;
+    pa.row_coef = W.row_coef;
+    pa.row_off = W.row_off;
+    pa.item_off_gu = W.item_gu;
+    pa.item_off_dn = W.item_dn;
+    pa.bn_gu = pa.bn_dn = plan.bn;
+    pa.mt_gu_routed = pa.mt_gu_shared = plan.pair ? H / 256 : H / 128;
+    pa.mt_dn = plan.pair ? d / 512 : (d + 255) / 256;
+    const cudaError_t ep = plan.permute_multi ? launch_permute_multi(pa, W.hist, s) : launch_permute(pa, s);
+    if (ep != cudaSuccess) return MOE_ERR_CUDA;
+    return run_experts(&c, wl, W, plan, di, n_rows, x_rows, false, y_rows, MOE_F32, 0, nullptr, s, nullptr, 1);
+}
+
+moe_status moe_ep_combine(int T, int d, int n_rows, const float* back_rows, const int32_t* send_tok, float* y_acc,
+                          void* y, const void* residual, moe_stream_t stream) {
+    if (T < 0 || d <= 0 || d % 8 != 0 || n_rows < 0) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return n_rows == 0 ? MOE_OK : MOE_ERR_INVALID_ARG;
+    if (!y_acc || !aligned16(y_acc) || (n_rows > 0 && (!back_rows || !send_tok || !aligned16(back_rows))) ||
+        (y && !aligned16(y)) || (residual && !aligned16(residual)))
+        return MOE_ERR_INVALID_ARG;
+    DevInfo di;
+    moe_status st = check_device(&di);
+    if (st != MOE_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (launch_ep_combine(back_rows, send_tok, n_rows, T, d, y_acc, di.sm_count, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (y && launch_finalize_bf16(y_acc, static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(y),
+                                  (size_t)T * d, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
 }
 
 }  // extern "C"

@@ -234,6 +234,13 @@ __device__ int block_excl_scan(int* a, int n, int* wsum) {
     return total;
 }
 
+// Group of global expert id `gid` when the groups are experts [lo, lo + E), else -1
+// (unsigned arithmetic: any int id, however negative, maps outside).
+__device__ __forceinline__ int local_expert(int gid, int lo, int E) {
+    const unsigned e = (unsigned)gid - (unsigned)lo;
+    return e < (unsigned)E ? (int)e : -1;
+}
+
 __global__ void __launch_bounds__(PERM_THREADS, 1) permute_kernel(PermuteArgs a, int WR) {
     extern __shared__ int psm[];
     const int E = a.E, T = a.T, k = a.k;
@@ -250,11 +257,11 @@ __global__ void __launch_bounds__(PERM_THREADS, 1) permute_kernel(PermuteArgs a,
     __syncthreads();
     bool bad = false;
     for (int p = tid; p < total_pairs; p += PERM_THREADS) {
-        int e = a.idx[p];
+        int e = local_expert(a.idx[p], a.id_lo, E);
         if (e >= 0 && e < E) atomicAdd(&s_scan[e], 1);
         else bad = true;
     }
-    if (bad) set_dev_error(MOE_DEVERR_BAD_EXPERT);
+    if (bad && !a.foreign_ok) set_dev_error(MOE_DEVERR_BAD_EXPERT);
     __syncthreads();
     for (int e = tid; e < E; e += PERM_THREADS) a.counts[e] = s_scan[e];
     __syncthreads();
@@ -301,7 +308,7 @@ __global__ void __launch_bounds__(PERM_THREADS, 1) permute_kernel(PermuteArgs a,
         const bool mine = warp < WR && t < T;
         if (mine) {
             for (int j = 0; j < k; ++j) {
-                int e = a.idx[(size_t)t * k + j];
+                int e = local_expert(a.idx[(size_t)t * k + j], a.id_lo, E);
                 if (e >= 0 && e < E) atomicOr(&s_mask[warp * E + e], 1u << lane);
             }
         }
@@ -319,7 +326,7 @@ __global__ void __launch_bounds__(PERM_THREADS, 1) permute_kernel(PermuteArgs a,
             const unsigned lower = (1u << lane) - 1u;
             for (int j = 0; j < k; ++j) {
                 const int p = t * k + j;
-                int e = a.idx[p];
+                int e = local_expert(a.idx[p], a.id_lo, E);
                 if (e >= 0 && e < E) {
                     int row = s_wbase[warp * E + e] + __popc(s_mask[warp * E + e] & lower);
                     a.src[row] = p;
@@ -356,11 +363,11 @@ __device__ __forceinline__ void build_lane_masks(const PermuteArgs& a, unsigned*
     if (t < a.T) {
         bool bad = false;
         for (int j = 0; j < k; ++j) {
-            const int e = a.idx[(size_t)t * k + j];
+            const int e = local_expert(a.idx[(size_t)t * k + j], a.id_lo, E);
             if (e >= 0 && e < E) atomicOr(&s_mask[warp * E + e], 1u << lane);
             else bad = true;
         }
-        if (bad && flag_bad) set_dev_error(MOE_DEVERR_BAD_EXPERT);
+        if (bad && flag_bad && !a.foreign_ok) set_dev_error(MOE_DEVERR_BAD_EXPERT);
     }
     __syncthreads();
 }
@@ -438,7 +445,7 @@ __global__ void __launch_bounds__(PERM_TB) permute_scatter_kernel(PermuteArgs a,
         const unsigned lower = (1u << lane) - 1u;
         for (int j = 0; j < k; ++j) {
             const int p = t * k + j;
-            const int e = a.idx[p];
+            const int e = local_expert(a.idx[p], a.id_lo, E);
             if (e >= 0 && e < E) {
                 const int row = s_wbase[warp * E + e] + __popc(s_mask[warp * E + e] & lower);
                 a.src[row] = p;
@@ -692,6 +699,117 @@ __global__ void __launch_bounds__(256) finalize_kernel(const float* __restrict__
             p[j] = *reinterpret_cast<uint32_t*>(&h);
         }
         *yp = make_uint4(p[0], p[1], p[2], p[3]);
+    }
+}
+
+// ============================================================================ expert parallelism
+// The experts are split over R ranks in contiguous blocks of epr = E / R; with
+// R = n_groups rank r holds group r (the pages' device-aligned groups).
+// Dispatch: token t goes to rank r when one of its k experts lies in r's block,
+// once per rank however many of its experts sit there.  Send rows are
+// rank-major, ascending token inside a rank.
+constexpr int EP_THREADS = 1024;
+
+__device__ __forceinline__ uint32_t ep_rank_mask(const int32_t* __restrict__ idx, int t, int k, int E, int epr) {
+    uint32_t m = 0;
+    for (int j = 0; j < k; ++j) {
+        const int e = idx[(size_t)t * k + j];
+        if ((unsigned)e < (unsigned)E) m |= 1u << (e / epr);
+    }
+    return m;
+}
+
+// one CTA per rank: the number of tokens it receives from this rank
+__global__ void __launch_bounds__(EP_THREADS) ep_count_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
+                                                              int epr, int32_t* __restrict__ counts) {
+    __shared__ int wsum[EP_THREADS / 32];
+    const int r = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int c = 0;
+    for (int t = threadIdx.x; t < T; t += EP_THREADS) c += (ep_rank_mask(idx, t, k, E, epr) >> r) & 1u;
+    for (int o = 16; o >= 1; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    if (lane == 0) wsum[warp] = c;
+    __syncthreads();
+    if (warp == 0) {
+        c = wsum[lane];
+        for (int o = 16; o >= 1; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+        if (lane == 0) counts[r] = c;
+    }
+}
+
+// one CTA per rank: its offset and its send rows' origin tokens, in token order
+__global__ void __launch_bounds__(EP_THREADS) ep_place_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
+                                                              int epr, int R, const int32_t* __restrict__ counts,
+                                                              int32_t* __restrict__ offsets,
+                                                              int32_t* __restrict__ send_tok) {
+    __shared__ int wsum[EP_THREADS / 32 + 1];
+    __shared__ int base_s;
+    const int r = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) {
+        int o = 0;
+        for (int q = 0; q < r; ++q) o += counts[q];
+        base_s = o;
+        offsets[r] = o;
+        if (r == R - 1) offsets[R] = o + counts[r];
+    }
+    __syncthreads();
+    int base = base_s;
+    for (int t0 = 0; t0 < T; t0 += EP_THREADS) {
+        const int t = t0 + threadIdx.x;
+        const bool mine = t < T && ((ep_rank_mask(idx, t, k, E, epr) >> r) & 1u);
+        const unsigned b = __ballot_sync(0xffffffffu, mine);
+        if (lane == 0) wsum[warp] = __popc(b);
+        __syncthreads();
+        if (warp == 0) {  // exclusive prefix over the 32 warps; wsum[32] = the chunk's total
+            const int v = wsum[lane];
+            int inc = v;
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += u;
+            }
+            wsum[lane] = inc - v;
+            if (lane == 31) wsum[32] = inc;
+        }
+        __syncthreads();
+        if (mine) send_tok[base + wsum[warp] + __popc(b & ((1u << lane) - 1u))] = t;
+        base += wsum[32];
+        __syncthreads();
+    }
+}
+
+// the routing of every send row: its token's k expert ids and weights
+__global__ void __launch_bounds__(256) ep_rows_kernel(const int32_t* __restrict__ idx, const float* __restrict__ w,
+                                                      int k, const int32_t* __restrict__ send_tok,
+                                                      const int32_t* __restrict__ n_rows_dev,
+                                                      int32_t* __restrict__ send_idx, float* __restrict__ send_w) {
+    const int n = *n_rows_dev * k;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+        const int r = i / k, j = i - r * k;
+        const size_t p = (size_t)send_tok[r] * k + j;
+        send_idx[i] = idx[p];
+        send_w[i] = w[p];
+    }
+}
+
+// combine: acc[send_tok[r], :] += back[r, :] (the partial sums the ranks returned)
+__global__ void __launch_bounds__(256) ep_combine_kernel(const float* __restrict__ back,
+                                                         const int32_t* __restrict__ send_tok, int n_rows, int T,
+                                                         int d, float* __restrict__ acc) {
+    const int d4 = d / 4;
+    const size_t n = (size_t)n_rows * d4;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        const size_t r = i / d4;
+        const int c = (int)(i - r * d4) * 4;
+        const int t = send_tok[r];
+        if ((unsigned)t >= (unsigned)T) {  // not a token of this batch: flagged and skipped
+            set_dev_error(MOE_DEVERR_BAD_ROWS);
+            continue;
+        }
+        const float4 v = *reinterpret_cast<const float4*>(back + r * d + c);
+        float* dst = acc + (size_t)t * d + c;
+        atomicAdd(dst + 0, v.x);
+        atomicAdd(dst + 1, v.y);
+        atomicAdd(dst + 2, v.z);
+        atomicAdd(dst + 3, v.w);
     }
 }
 
@@ -987,6 +1105,36 @@ cudaError_t read_clear_dev_error(unsigned int* flags, cudaStream_t s) {
                    cudaSuccess
                ? cudaStreamSynchronize(s)
                : cudaGetLastError();
+}
+
+cudaError_t launch_ep_dispatch(const int32_t* idx, const float* w, int T, int k, int E, int R, const void* x,
+                               bool x_f32, int d, int32_t* counts, int32_t* offsets, int32_t* send_tok,
+                               __nv_bfloat16* send_x, int32_t* send_idx, float* send_w, int n_sm, cudaStream_t s) {
+    const int epr = E / R;
+    note_launch();
+    ep_count_kernel<<<R, EP_THREADS, 0, s>>>(idx, T, k, E, epr, counts);
+    note_launch();
+    ep_place_kernel<<<R, EP_THREADS, 0, s>>>(idx, T, k, E, epr, R, counts, offsets, send_tok);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || T == 0) return e;
+    const int max_rows = T * (k < R ? k : R);
+    if ((e = launch_gather(x, x_f32, d, send_tok, offsets + R, max_rows, send_x, n_sm, s)) != cudaSuccess) return e;
+    int grid = (max_rows * k + 255) / 256;
+    grid = grid < n_sm * 4 ? grid : n_sm * 4;
+    note_launch();
+    ep_rows_kernel<<<grid, 256, 0, s>>>(idx, w, k, send_tok, offsets + R, send_idx, send_w);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ep_combine(const float* back, const int32_t* send_tok, int n_rows, int T, int d, float* acc,
+                              int n_sm, cudaStream_t s) {
+    if (n_rows == 0) return cudaSuccess;
+    const size_t n = (size_t)n_rows * (d / 4);
+    size_t grid = (n + 255) / 256;
+    if (grid > (size_t)n_sm * 16) grid = (size_t)n_sm * 16;
+    note_launch();
+    ep_combine_kernel<<<(unsigned)grid, 256, 0, s>>>(back, send_tok, n_rows, T, d, acc);
+    return cudaGetLastError();
 }
 
 }  // namespace moe

@@ -52,6 +52,10 @@ enum { MODE_GATEUP = 0, MODE_DOWN = 1, MODE_LOGITS = 2 };
 struct PermuteArgs {
     const int32_t* idx;
     int T, k, E;
+    // expert id e of a pair maps to group e - id_lo; ids outside [id_lo, id_lo + E)
+    // are errors (MOE_DEVERR_BAD_EXPERT), or with foreign_ok another rank's experts
+    // that this call skips silently
+    int id_lo, foreign_ok;
     int32_t* counts;   // [E]
     int32_t* offsets;  // [E + 1]
     int32_t* src;      // [T * k]
@@ -83,6 +87,16 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
 // Forward mode only, many CTAs: needs hist [permute_blocks(T) * E] int32 of scratch.
 int permute_blocks(int T);
 cudaError_t launch_permute_multi(const PermuteArgs& a, int32_t* hist, cudaStream_t s);
+// Expert parallelism over R ranks (contiguous blocks of E / R experts, R <= 32):
+// counts[R], offsets[R + 1], and per send row (rank-major, ascending token) its
+// origin token, x row (bf16) and the token's k expert ids and weights.
+cudaError_t launch_ep_dispatch(const int32_t* idx, const float* w, int T, int k, int E, int R, const void* x,
+                               bool x_f32, int d, int32_t* counts, int32_t* offsets, int32_t* send_tok,
+                               __nv_bfloat16* send_x, int32_t* send_idx, float* send_w, int n_sm, cudaStream_t s);
+// acc[send_tok[r], :] += back[r, :] for r < n_rows (fp32 atomics; d % 4 == 0); a token
+// outside [0, T) sets MOE_DEVERR_BAD_ROWS and its row is skipped
+cudaError_t launch_ep_combine(const float* back, const int32_t* send_tok, int n_rows, int T, int d, float* acc,
+                              int n_sm, cudaStream_t s);
 // x_perm[r, :] = x[row_tok[r], :] (fp32 input rounded to bf16) for r < row_off[n_groups]
 cudaError_t launch_gather(const void* x, bool x_f32, int d, const int32_t* row_tok, const int32_t* n_rows_dev,
                           int max_rows, __nv_bfloat16* x_perm, int n_sm, cudaStream_t s);

@@ -1,0 +1,105 @@
+"""Expert parallelism: the MoE layer forward with the routed experts split over the
+ranks of a process group (one process per GPU) in contiguous blocks of E / world
+experts.  With world = n_groups each rank holds one group of 32 experts: the
+groups are device-aligned ("DeepSeek-V3" llm-vis, "MoE router" box), so a token's
+rows go to at most topk_groups ranks.
+
+One forward on every rank, in the same order on all of them:
+
+    moe_route         own tokens -> topk_idx, topk_w
+    moe_ep_dispatch   rows for each rank (each token once per rank), rank-major
+    exchange          counts, then rows, expert ids and weights (all-to-all)
+    moe_experts_routed  this rank's block of experts on the rows it received
+    exchange          the fp32 partial sums back to the ranks the rows came from
+    moe_dense_ffn     the shared expert on own tokens, fp32 (y_acc)
+    moe_ep_combine    y_acc[token] += partial sums; y = bf16(y_acc)
+
+Every step but the exchange runs in the library's kernels; the exchange is
+torch.distributed's all-to-all (NCCL between GPUs, gloo on CPU).  The result
+equals moe_forward's on the same tokens up to the order of fp32 additions.
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+from . import (MOE_BF16, MOE_E4M3, MoeConfig, dense_workspace_size, ep_max_send_rows, experts_routed_workspace_size,
+               moe_dense_ffn, moe_ep_combine, moe_ep_dispatch, moe_experts_routed, moe_route)
+
+
+def exchange_counts(send_counts: torch.Tensor, group=None) -> torch.Tensor:
+    """send_counts[q] = rows this rank sends to rank q; returns recv_counts[q] = rows rank q sends here."""
+    recv = torch.empty_like(send_counts)
+    dist.all_to_all_single(recv, send_counts, group=group)
+    return recv
+
+
+def exchange(send: torch.Tensor, send_counts: list[int], recv_counts: list[int], group=None) -> torch.Tensor:
+    """Rows of ``send`` (rank-major: send_counts[q] rows for rank q) to their ranks; returns the rows this rank
+    receives, rank-major (recv_counts[q] rows from rank q)."""
+    recv = send.new_empty((sum(recv_counts),) + tuple(send.shape[1:]))
+    dist.all_to_all_single(recv, send[: sum(send_counts)].contiguous(), recv_counts, send_counts, group=group)
+    return recv
+
+
+def expert_block(cfg: MoeConfig, rank: int, world: int) -> tuple[int, int]:
+    """(first expert, number of experts) of ``rank``'s block."""
+    if cfg.n_experts % world:
+        raise ValueError(f"{cfg.n_experts} experts do not split over {world} ranks")
+    n = cfg.n_experts // world
+    return rank * n, n
+
+
+def moe_forward_ep(cfg: MoeConfig, w_router, local_weights: dict, shared_weights: dict, bias, x, y, group=None,
+                   residual=None):
+    """y = MoE(x) (+ residual) for this rank's tokens x [T, d], with this rank's block of experts.
+
+    ``local_weights``: the block's w_gate / w_up [n, H, d], w_down [n, d, H] (e4m3: plus s_gate / s_up / s_down),
+    n = E / world.  ``shared_weights``: the shared expert's w_gate / w_up [Hs, d], w_down [d, Hs] (e4m3: plus
+    their scales).  ``y`` [T, d] bf16 (may be ``residual``).  Every rank of ``group`` calls this together.  The
+    kernels run on the current stream, which torch.distributed orders the collectives with."""
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    lo, n_local = expert_block(cfg, rank, world)
+    if cfg.n_shared != 1:
+        raise ValueError("the expert-parallel layer takes one shared expert")
+    dev = x.device
+    T, d, k = x.shape[0], cfg.d, cfg.top_k
+    # (1) routing of this rank's tokens
+    logits = torch.empty((T, cfg.n_experts), dtype=torch.float32, device=dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    moe_route(cfg, x, w_router, logits, bias, idx, w)
+    # (2) dispatch
+    rows = ep_max_send_rows(cfg, T, world)
+    counts = torch.empty(world, dtype=torch.int32, device=dev)
+    offsets = torch.empty(world + 1, dtype=torch.int32, device=dev)
+    send_tok = torch.empty(max(rows, 1), dtype=torch.int32, device=dev)
+    send_x = torch.empty((max(rows, 1), d), dtype=torch.bfloat16, device=dev)
+    send_idx = torch.empty((max(rows, 1), k), dtype=torch.int32, device=dev)
+    send_w = torch.empty((max(rows, 1), k), dtype=torch.float32, device=dev)
+    moe_ep_dispatch(cfg, world, idx, w, x, counts, offsets, send_tok, send_x, send_idx, send_w)
+    # (3) exchange: the split sizes must be known on the host
+    recv_counts = exchange_counts(counts, group)
+    sc, rc = counts.tolist(), recv_counts.tolist()
+    recv_x = exchange(send_x, sc, rc, group)
+    recv_idx = exchange(send_idx, sc, rc, group)
+    recv_w = exchange(send_w, sc, rc, group)
+    # (4) this rank's experts on the rows it received
+    n_recv = recv_x.shape[0]
+    recv_y = torch.empty((n_recv, d), dtype=torch.float32, device=dev)
+    if n_recv:
+        ws = torch.empty(experts_routed_workspace_size(cfg, n_local, n_recv), dtype=torch.uint8, device=dev)
+        moe_experts_routed(cfg, local_weights, lo, n_local, recv_x, recv_idx, recv_w, recv_y, workspace=ws)
+    # (5) the partial sums back to where the rows came from
+    back = exchange(recv_y, rc, sc, group)
+    # (6) the shared expert on this rank's tokens, (7) combine
+    y_acc = torch.empty((T, d), dtype=torch.float32, device=dev)
+    if T:
+        wdt = MOE_E4M3 if shared_weights["w_gate"].dtype == torch.uint8 else MOE_BF16
+        hs = shared_weights["w_gate"].shape[0]
+        dws = torch.empty(dense_workspace_size(d, hs, cfg.act_dtype, wdt, T), dtype=torch.uint8, device=dev)
+        moe_dense_ffn(shared_weights["w_gate"], shared_weights["w_up"], shared_weights["w_down"], x, y_acc,
+                      shared_weights.get("s_gate"), shared_weights.get("s_up"), shared_weights.get("s_down"),
+                      workspace=dws)
+        moe_ep_combine(back, send_tok, y_acc, y, residual)

@@ -67,7 +67,7 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_E4M3 = 2 } moe_dtype;
 /* Device error word bits (moe_device_error). */
 #define MOE_DEVERR_BAD_EXPERT 0x1u    /* a routed expert id outside [0, n_experts) */
 #define MOE_DEVERR_TIMEOUT    0x2u    /* a pipeline wait exceeded its limit */
-#define MOE_DEVERR_BAD_ROWS   0x4u    /* a tile schedule entry outside its buffer */
+#define MOE_DEVERR_BAD_ROWS   0x4u    /* a schedule entry or a combine row's token outside its buffer */
 
 /* Layer shape ("Teardown: DeepSeek-V3", At a glance + section 6; field guide
  * cutaway 02).  Constraints checked by every entry point:
@@ -322,6 +322,68 @@ MOE_API moe_status moe_dense_ffn(int d, int hidden, moe_dtype act_dtype, moe_dty
                                  const float* s_down, const void* x, int T, void* y, moe_dtype y_dtype,
                                  int accumulate, void* workspace, size_t ws_bytes, moe_stream_t stream,
                                  const moe_stage_events* events);
+
+/* ---------------------------------------------------------------- expert parallelism
+ * The routed experts split over n_ranks ranks (one process per GPU) in
+ * contiguous blocks of E / n_ranks.  With n_ranks = n_groups rank r holds group
+ * r: the pages' groups are device-aligned ("DeepSeek-V3" llm-vis, "MoE router"
+ * box), so a token reaches at most topk_groups ranks.  One layer forward on a
+ * rank: moe_route on its own tokens -> moe_ep_dispatch -> all-to-all of the
+ * counts and the rows (the caller's collective, e.g. NCCL) -> moe_experts_routed
+ * on the received rows -> all-to-all of the results back -> the shared expert
+ * on the rank's own tokens (moe_dense_ffn into an fp32 y_acc) -> moe_ep_combine.
+ * The result equals moe_forward's up to the order of the fp32 additions. */
+
+/* Most send rows moe_ep_dispatch produces for T tokens: T * min(k, n_ranks)
+ * (0 on invalid arguments). */
+MOE_API int moe_ep_max_send_rows(const moe_config* cfg, int T, int n_ranks);
+
+/* Dispatch.  For each rank q = 0 .. n_ranks-1, the tokens with at least one of
+ * their k selected experts in q's block [q E/n_ranks, (q+1) E/n_ranks), each
+ * once, in ascending token order; the rows are rank-major:
+ *   topk_idx [T, k] int32, topk_w [T, k] fp32  moe_route's routing (ids outside
+ *                                              [0, E) are ignored)
+ *   x [T, d] cfg->act_dtype                    the rank's activations
+ *   send_counts [n_ranks], send_offsets [n_ranks + 1] (exclusive prefix sum;
+ *                                              send_offsets[n_ranks] = rows)
+ *   send_tok [rows]    origin token of each row
+ *   send_x [rows, d]   bf16 rows of x (fp32 x rounded to bf16, as the experts round it)
+ *   send_idx [rows, k], send_w [rows, k]  the token's whole routing (the
+ *                                         receiver keeps the slots of its block)
+ * The row arrays hold moe_ep_max_send_rows rows; counts and offsets are written
+ * for T = 0 too.  n_ranks in [1, 32] and dividing E; x and send_x 16-byte aligned. */
+MOE_API moe_status moe_ep_dispatch(const moe_config* cfg, int n_ranks, const int32_t* topk_idx, const float* topk_w,
+                                   const void* x, int T, int32_t* send_counts, int32_t* send_offsets,
+                                   int32_t* send_tok, void* send_x, int32_t* send_idx, float* send_w,
+                                   moe_stream_t stream);
+
+/* Device workspace bytes of moe_experts_routed for up to n_rows_max rows and a
+ * block of n_local experts (0 on invalid arguments). */
+MOE_API size_t moe_experts_routed_workspace_size(const moe_config* cfg, int n_local, int n_rows_max);
+
+/* The experts of one block on rows whose routing is given (the receiving side
+ * of the dispatch; "Routed experts" and "Expert combine" boxes):
+ *   y_rows[i] = routed_scale * sum over the slots j whose expert lies in
+ *               [expert_lo, expert_lo + n_local) of w[i,j] * expert_{idx[i,j]}(x_rows[i])
+ * fp32 [n_rows, d], overwritten; expert(x) and the arithmetic as moe_forward's.
+ * w_local: the block's weights, w_gate / w_up [n_local, H, d], w_down [n_local,
+ * d, H] (e4m3: with their block scales); its router and shared-expert pointers
+ * are not read.  x_rows [n_rows, d] bf16; topk_idx / topk_w [n_rows, k] with
+ * global expert ids (slots of other blocks are skipped, not errors).
+ * workspace: moe_experts_routed_workspace_size(cfg, n_local, n_rows) bytes,
+ * 256-byte aligned. */
+MOE_API moe_status moe_experts_routed(const moe_config* cfg, const moe_weights* w_local, int expert_lo, int n_local,
+                                      const void* x_rows, int n_rows, const int32_t* topk_idx, const float* topk_w,
+                                      float* y_rows, void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/* Combine: y_acc[send_tok[i], :] += back_rows[i, :] for i < n_rows (fp32
+ * atomics: a token's partial sums from its <= topk_groups ranks), then, with y
+ * not NULL, y = bf16(y_acc + residual) ([T, d] bf16; residual bf16 [T, d] or
+ * NULL, and may be y itself).  y_acc [T, d] fp32 holds the shared expert's output
+ * on entry.  A send_tok entry outside [0, T) sets MOE_DEVERR_BAD_ROWS and its
+ * row is skipped.  d a multiple of 8; arrays 16-byte aligned. */
+MOE_API moe_status moe_ep_combine(int T, int d, int n_rows, const float* back_rows, const int32_t* send_tok,
+                                  float* y_acc, void* y, const void* residual, moe_stream_t stream);
 
 /* Size of the device scratch array that moe_forward_noalloc uses in place of
  * a caller-provided workspace: 32 MiB.  At the DeepSeek-V3 sizes (d = 7168,

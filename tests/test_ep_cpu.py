@@ -1,0 +1,139 @@
+"""Expert parallelism on the CPU: the exchange protocol of moe_forward_ep with gloo
+ranks (world size 2 and 4), and the EP entry points' argument checks (no device).
+
+The exchange test runs the protocol moe_forward_ep runs (counts all-to-all, then
+rows, routing and results) on rows built by the dispatch's definition: for each
+destination rank the tokens with an expert in its block, ascending, rank-major.
+Each rank stands in for the expert kernels with a known map of the rows it
+received (row * (rank + 1) + slot count of its block), so a row that comes back
+from the wrong rank, in the wrong order or to the wrong token fails."""
+import ctypes
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import fine_grained_moe_gemm_b200 as moe
+from moe_testlib import cfg_of
+from workloads import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def dispatch_def(idx: np.ndarray, E: int, R: int):
+    """The dispatch by its definition: per destination rank the tokens with at least one expert in its block,
+    ascending; returns (counts, send_tok) with send_tok rank-major."""
+    epr = E // R
+    rows = [[t for t in range(idx.shape[0]) if any(0 <= e < E and e // epr == q for e in idx[t])] for q in range(R)]
+    return np.array([len(r) for r in rows], np.int32), np.array([t for r in rows for t in r], np.int32)
+
+
+def _rank_main(rank, world, port, out):
+    import datetime
+
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from fine_grained_moe_gemm_b200 import ep
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    E, k, T, d = 16, 4, 11 + 3 * rank, 8
+    rng = np.random.default_rng(100 + rank)
+    idx = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+    x = torch.from_numpy(rng.standard_normal((T, d)).astype(np.float32))
+    counts, send_tok = dispatch_def(idx, E, world)
+    send_x = x[torch.from_numpy(send_tok).long()]
+    send_idx = torch.from_numpy(idx[send_tok])
+    recv_counts = ep.exchange_counts(torch.from_numpy(counts), None)
+    sc, rc = counts.tolist(), recv_counts.tolist()
+    recv_x = ep.exchange(send_x, sc, rc)
+    recv_idx = ep.exchange(send_idx, sc, rc)
+    # stand-in for this rank's experts: a map the origin rank can predict
+    epr = E // world
+    mine = ((recv_idx >= rank * epr) & (recv_idx < (rank + 1) * epr)).sum(1, keepdim=True).float()
+    recv_y = recv_x * (rank + 1) + mine
+    back = ep.exchange(recv_y, rc, sc)
+    # the rows came back in send order: row i is token send_tok[i] after rank q's map
+    ok = True
+    base = 0
+    for q in range(world):
+        for i in range(base, base + sc[q]):
+            t = send_tok[i]
+            n_q = int(((idx[t] >= q * epr) & (idx[t] < (q + 1) * epr)).sum())
+            ok &= n_q > 0 and torch.equal(back[i], x[t] * (q + 1) + n_q)
+        base += sc[q]
+    total = torch.tensor([int(recv_counts.sum())])
+    dist.all_reduce(total)
+    dist.barrier()
+    dist.destroy_process_group()
+    with open(os.path.join(out, f"r{rank}"), "w") as f:
+        f.write(f"{int(ok)} {int(counts.sum())} {int(total)}")
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_exchange_protocol_gloo(tmp_path, world):
+    port = _free_port()
+    mp.spawn(_rank_main, args=(world, port, str(tmp_path)), nprocs=world, join=True)
+    res = [open(tmp_path / f"r{r}").read().split() for r in range(world)]
+    assert all(r[0] == "1" for r in res)
+    # every row sent was received: the sum of the ranks' send rows = the rows all ranks received
+    assert sum(int(r[1]) for r in res) == int(res[0][2])
+
+
+def test_dispatch_definition_bounds():
+    """A token reaches at most min(k, ranks) ranks, and with ranks = groups at most topk_groups of them
+    when its experts come from topk_groups groups."""
+    E, G, k = 256, 8, 8
+    rng = np.random.default_rng(0)
+    groups = [rng.choice(G, 4, replace=False) for _ in range(64)]
+    idx = np.stack([np.concatenate([rng.choice(32, 2, replace=False) + 32 * g for g in gs]) for gs in groups])
+    counts, tok = dispatch_def(idx.astype(np.int32), E, G)
+    per_token = np.bincount(tok, minlength=64)
+    assert per_token.max() <= 4 and per_token.min() >= 1 and counts.sum() == per_token.sum()
+
+
+@pytest.fixture(scope="module")
+def L():
+    return moe.lib()
+
+
+def test_ep_entry_arguments(L):
+    cfg = cfg_of(WORKLOADS["decode"])
+    P = ctypes.c_void_p
+    assert L.moe_ep_max_send_rows(ctypes.byref(cfg), 128, 8) == 128 * 8
+    assert L.moe_ep_max_send_rows(ctypes.byref(cfg), 128, 4) == 128 * 4
+    assert L.moe_ep_max_send_rows(ctypes.byref(cfg), 128, 0) == 0
+    disp = lambda R, counts: L.moe_ep_dispatch(ctypes.byref(cfg), R, P(16), P(16), P(16), 4, counts, P(16), P(16),
+                                               P(16), P(16), P(16), None)
+    assert disp(0, P(16)) == moe.MOE_ERR_INVALID_ARG          # no ranks
+    assert disp(33, P(16)) == moe.MOE_ERR_INVALID_ARG         # more than 32
+    assert disp(3, P(16)) == moe.MOE_ERR_INVALID_ARG          # 256 experts do not split over 3
+    assert disp(8, None) == moe.MOE_ERR_INVALID_ARG           # no counts
+    assert L.moe_ep_dispatch(ctypes.byref(cfg), 8, P(16), P(16), P(18), 4, P(16), P(16), P(16), P(16), P(16), P(16),
+                             None) == moe.MOE_ERR_INVALID_ARG  # misaligned x
+    # the block computation: block inside [0, E), enough workspace
+    assert L.moe_experts_routed_workspace_size(ctypes.byref(cfg), 32, 1024) > 0
+    assert L.moe_experts_routed_workspace_size(ctypes.byref(cfg), 0, 1024) == 0
+    w = moe.MoeWeights(w_gate=16, w_up=16, w_down=16)
+    er = lambda lo, n, ws: L.moe_experts_routed(ctypes.byref(cfg), ctypes.byref(w), lo, n, P(16), 4, P(16), P(16),
+                                                P(16), P(1 << 20), ws, None)
+    assert er(240, 32, 1 << 30) == moe.MOE_ERR_INVALID_ARG   # past the last expert
+    assert er(-1, 32, 1 << 30) == moe.MOE_ERR_INVALID_ARG
+    assert er(0, 32, 1024) == moe.MOE_ERR_WORKSPACE
+    assert L.moe_experts_routed(ctypes.byref(cfg), ctypes.byref(w), 0, 32, P(16), 0, None, None, None, None, 0,
+                                None) == moe.MOE_OK           # no rows: a no-op
+    # the combine
+    assert L.moe_ep_combine(4, 7164, 2, P(16), P(16), P(16), None, None, None) == moe.MOE_ERR_INVALID_ARG  # d % 8
+    assert L.moe_ep_combine(4, 7168, 2, P(16), P(16), None, None, None, None) == moe.MOE_ERR_INVALID_ARG  # no y_acc
+    assert L.moe_ep_combine(0, 7168, 0, None, None, None, None, None, None) == moe.MOE_OK
+    assert L.moe_ep_combine(0, 7168, 3, None, None, None, None, None, None) == moe.MOE_ERR_INVALID_ARG
