@@ -218,3 +218,34 @@ def test_forward_ep_one_rank_nccl():
     # one bf16 rounding (half an ulp of |ref|, up to 2^-8 |ref|) away from a value close to ref
     rms = float(ref.double().pow(2).mean().sqrt())
     assert bool(((y.double() - ref.double()).abs() <= 2.0 ** -8 * ref.double().abs() + 1e-3 * rms).all())
+
+
+def test_combine_flags_a_token_outside_the_batch():
+    """A returned row whose token is not in the batch is skipped and flagged (MOE_DEVERR_BAD_ROWS) by the
+    kernel's bounds check; the other rows land."""
+    T, d = 4, 256
+    y_acc = torch.zeros((T, d), dtype=torch.float32, device=DEV)
+    back = torch.arange(3 * d, dtype=torch.float32, device=DEV).reshape(3, d)
+    tok = torch.tensor([0, 7, 2], dtype=torch.int32, device=DEV)
+    y = torch.empty((T, d), dtype=torch.bfloat16, device=DEV)
+    moe.moe_ep_combine(back, tok, y_acc, y)
+    torch.cuda.synchronize()
+    assert moe.device_error() == moe.MOE_DEVERR_BAD_ROWS
+    expect = torch.zeros((T, d), dtype=torch.float32, device=DEV)
+    expect[0], expect[2] = back[0], back[2]
+    assert torch.equal(y_acc, expect)
+    assert torch.equal(y, expect.to(torch.bfloat16))
+
+
+def test_dispatch_of_no_tokens_writes_zero_counts():
+    wl, W = inputs("decode")
+    cfg = cfg_of(wl)
+    R = 8
+    counts = torch.full((R,), -1, dtype=torch.int32, device=DEV)
+    offsets = torch.full((R + 1,), -1, dtype=torch.int32, device=DEV)
+    e = lambda *shape, dt=torch.int32: torch.empty(shape, dtype=dt, device=DEV)
+    moe.moe_ep_dispatch(cfg, R, e(0, wl.top_k), e(0, wl.top_k, dt=torch.float32), e(0, wl.d, dt=torch.bfloat16),
+                        counts, offsets, e(1), e(1, wl.d, dt=torch.bfloat16), e(1, wl.top_k),
+                        e(1, wl.top_k, dt=torch.float32))
+    torch.cuda.synchronize()
+    assert counts.tolist() == [0] * R and offsets.tolist() == [0] * (R + 1)
