@@ -377,7 +377,7 @@ MOE_API moe_status moe_experts_routed(const moe_config* cfg, const moe_weights* 
                                       float* y_rows, void* workspace, size_t ws_bytes, moe_stream_t stream);
 
 /* Combine: y_acc[send_tok[i], :] += back_rows[i, :] for i < n_rows (fp32
- * atomics: a token's partial sums from its <= topk_groups ranks), then, with y
+ * atomics: a token's partial sums from the ranks it was sent to), then, with y
  * not NULL, y = bf16(y_acc + residual) ([T, d] bf16; residual bf16 [T, d] or
  * NULL, and may be y itself).  y_acc [T, d] fp32 holds the shared expert's output
  * on entry.  A send_tok entry outside [0, T) sets MOE_DEVERR_BAD_ROWS and its
