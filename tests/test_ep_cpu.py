@@ -137,3 +137,90 @@ def test_ep_entry_arguments(L):
     assert L.moe_ep_combine(4, 7168, 2, P(16), P(16), None, None, None, None) == moe.MOE_ERR_INVALID_ARG  # no y_acc
     assert L.moe_ep_combine(0, 7168, 0, None, None, None, None, None, None) == moe.MOE_OK
     assert L.moe_ep_combine(0, 7168, 3, None, None, None, None, None, None) == moe.MOE_ERR_INVALID_ARG
+
+
+# ----------------------------------------------------------------------------- moe_forward_ep's control flow
+# The real moe_forward_ep runs on gloo ranks with the library calls replaced by CPU stand-ins of known
+# arithmetic (routing: the top-k of the first E features; expert e: x -> (e + 1) x; shared: x -> x / 2),
+# so each token's output has a closed form: bf16(x/2 + 2.5 * sum_j w_j (idx_j + 1) x).  A row sent to
+# the wrong rank, a slot counted twice or dropped, or a result combined into the wrong token fails.
+
+def _stand_ins(ep_mod, E_total):
+    def route(cfg, x, w_router, logits, bias, idx, w, stream=None):
+        s = x.float()[:, :cfg.n_experts]
+        top = torch.topk(s, cfg.top_k, dim=1)
+        idx.copy_(top.indices.to(torch.int32))
+        p = torch.sigmoid(top.values)
+        w.copy_(p / p.sum(1, keepdim=True))
+
+    def dispatch(cfg, R, idx, w, x, counts, offsets, send_tok, send_x, send_idx, send_w, stream=None):
+        c, tok = dispatch_def(idx.numpy(), cfg.n_experts, R)
+        counts.copy_(torch.from_numpy(c))
+        offsets.copy_(torch.from_numpy(np.concatenate([[0], np.cumsum(c)]).astype(np.int32)))
+        n = len(tok)
+        t = torch.from_numpy(tok).long()
+        send_tok[:n] = t.to(torch.int32)
+        send_x[:n] = x[t].to(send_x.dtype)
+        send_idx[:n] = idx[t]
+        send_w[:n] = w[t]
+
+    def experts(cfg, local_weights, lo, n, x_rows, idx, w, y_rows, workspace=None, stream=None):
+        mine = (idx >= lo) & (idx < lo + n)
+        coef = (w * (idx.float() + 1) * mine.float()).sum(1, keepdim=True)
+        y_rows.copy_(cfg.routed_scale * coef * x_rows.float())
+
+    def dense(wg, wu, wd, x, y, *a, **k):
+        y.copy_(0.5 * x.float())
+
+    def combine(back, send_tok, y_acc, y=None, residual=None, stream=None):
+        y_acc.index_add_(0, send_tok[: back.shape[0]].long(), back)
+        if y is not None:
+            y.copy_((y_acc + (residual.float() if residual is not None else 0)).to(torch.bfloat16))
+
+    ep_mod.moe_route, ep_mod.moe_ep_dispatch, ep_mod.moe_experts_routed = route, dispatch, experts
+    ep_mod.moe_dense_ffn, ep_mod.moe_ep_combine = dense, combine
+    ep_mod.ep_max_send_rows = lambda cfg, T, R: T * min(cfg.top_k, R)
+    ep_mod.experts_routed_workspace_size = lambda cfg, n, rows: 1
+    ep_mod.dense_workspace_size = lambda *a: 1
+
+
+def _forward_rank(rank, world, port, out):
+    import datetime
+
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import fine_grained_moe_gemm_b200 as moe_pkg
+    from fine_grained_moe_gemm_b200 import ep
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    E, k, d = 16, 4, 32
+    cfg = moe_pkg.MoeConfig(d * 4, E, 4, 2, k, 128, 1, 128, 2.5)  # d field unused by the stand-ins
+    cfg.d = d
+    _stand_ins(ep, E)
+    T = 9 + 5 * rank
+    g = torch.Generator().manual_seed(7 + rank)
+    x = torch.randn((T, d), generator=g).to(torch.bfloat16)
+    y = torch.empty((T, d), dtype=torch.bfloat16)
+    shared = {n: torch.empty((128, d), dtype=torch.bfloat16) for n in ("w_gate", "w_up", "w_down")}
+    ep.moe_forward_ep(cfg, None, {}, shared, torch.zeros(E), x, y)
+    # the closed form per token
+    xf = x.double()
+    top = torch.topk(xf.float()[:, :E], k, dim=1)
+    p = torch.sigmoid(top.values)
+    wts = (p / p.sum(1, keepdim=True)).double()
+    coef = (wts * (top.indices.double() + 1)).sum(1, keepdim=True)
+    ref = 0.5 * xf + 2.5 * coef * xf
+    ulp = 2.0 ** -7 * ref.abs() + 1e-6
+    ok = bool(((y.double() - ref).abs() <= ulp).all())
+    dist.barrier()
+    dist.destroy_process_group()
+    with open(os.path.join(out, f"f{rank}"), "w") as f:
+        f.write(str(int(ok)))
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_forward_ep_control_flow_gloo(tmp_path, world):
+    port = _free_port()
+    mp.spawn(_forward_rank, args=(world, port, str(tmp_path)), nprocs=world, join=True)
+    assert all(open(tmp_path / f"f{r}").read() == "1" for r in range(world))
