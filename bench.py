@@ -6,7 +6,14 @@ One step = one moe_forward (router, group-limited top-8 selection, permutation,
 batch of T tokens whose inputs are already resident in HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|skewed|fp8|tiny]
+                    [--op layer|block|dense]
     python bench.py --impl reference ...   # the CPU oracle on a bounded sample
+
+`value` times the step alone (CUDA-graph replay, or eager steps with an L2 flush
+for inputs that fit in L2); `e2e` times it with host buffers, the copy of x in
+and of y out inside every step, through the C ABI's host-buffer entry point:
+`e2e.value` with the steps alternating between two streams (one step's copies
+overlap the other's kernels), `e2e.serial_value` one step after another.
 
 With N > 1 (launched by torchrun) every rank runs an independent replica of
 the layer on its own GPU and batch (weak scaling; the layer has no exchange
