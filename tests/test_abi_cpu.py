@@ -175,3 +175,22 @@ def test_host_entry_arguments(L):
     nodev = L.moe_forward_host(ctypes.byref(cfg), ctypes.byref(moe.MoeWeights()), P(17), P(16), 4, P(19),
                                moe.MOE_BF16, 0, P(1 << 20), 1 << 30, None)
     assert nodev == moe.MOE_ERR_INVALID_ARG                                              # no weights
+
+
+def test_binding_argument_counts_match_the_header(L):
+    """Every entry point the binding declares argument types for takes as many parameters as its
+    declaration in include/moe.h (a drift between the two would pass wrong values silently)."""
+    import re
+    text = open(moe.HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    decls = dict(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(([^)]*)\)\s*;", text))
+    assert set(decls) == set(moe.declared_symbols())
+    checked = 0
+    for name, params in decls.items():
+        argtypes = getattr(L, name).argtypes
+        if argtypes is None:
+            continue
+        n = 0 if params.strip() in ("", "void") else params.count(",") + 1
+        assert len(argtypes) == n, f"{name}: header {n} parameters, binding {len(argtypes)}"
+        checked += 1
+    assert checked >= 20
