@@ -26,7 +26,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "moe.h")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_DEVICE, MOE_ERR_CUDA = range(6)
 MOE_F32, MOE_BF16, MOE_E4M3 = 0, 1, 2
-MOE_DEVERR_BAD_EXPERT, MOE_DEVERR_TIMEOUT, MOE_DEVERR_BAD_ROWS = 1, 2, 4
+MOE_DEVERR_BAD_EXPERT, MOE_DEVERR_TIMEOUT, MOE_DEVERR_BAD_ROWS, MOE_DEVERR_NONFINITE = 1, 2, 4, 8
 
 _lib = None
 _lock = threading.Lock()

@@ -122,6 +122,12 @@ __global__ void __launch_bounds__(SELECT_THREADS) select_kernel(float* __restric
         float sv = sigmoid_spec(lv);
         float bv = __fadd_rn(sv, bias[e]);
         if (bv == 0.0f) bv = 0.0f;
+        if (!isfinite(lv) || bv != bv) {
+            // logits must be finite: flag it, and let a NaN rank last so every
+            // decision below still picks valid ids
+            set_dev_error(MOE_DEVERR_NONFINITE);
+            if (bv != bv) bv = -INFINITY;
+        }
         ssm[(size_t)tl * 2 * E + e] = sv;
         ssm[(size_t)tl * 2 * E + E + e] = bv;
     }
@@ -145,14 +151,16 @@ __global__ void __launch_bounds__(SELECT_THREADS) select_kernel(float* __restric
         }
         gsc = __fadd_rn(b[i1], b[i2]);
         if (gsc == 0.0f) gsc = 0.0f;
+        if (gsc != gsc) gsc = -INFINITY;
     }
     unsigned gmask = 0;
     for (int r = 0; r < topk_groups; ++r) {
+        // non-candidates carry id G: any candidate, even at -inf, ranks before them
         bool cand = lane < G && !((gmask >> lane) & 1u);
         float v = cand ? gsc : -INFINITY;
-        int id = cand ? lane : 0x7fffffff;
+        int id = cand ? lane : G;
         warp_best(v, id);
-        gmask |= 1u << id;
+        if (id < G) gmask |= 1u << id;
     }
     // experts: lane owns e = lane + 32 i
     unsigned taken = 0;
@@ -167,8 +175,8 @@ __global__ void __launch_bounds__(SELECT_THREADS) select_kernel(float* __restric
             }
         }
         warp_best(v, id);
-        if ((id & 31) == lane) taken |= 1u << (id >> 5);
-        if (lane == j) my_idx = id;
+        if (id < E && (id & 31) == lane) taken |= 1u << (id >> 5);
+        if (lane == j) my_idx = id < E ? id : 0;
     }
     // S over the selected experts in ascending expert index
     int rank = 0;

@@ -19,15 +19,28 @@ std::mutex g_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the scratch on the current device (looked up once per
-// device, with that device current).
+// device, with that device current).  A device that is not sm_100 is refused
+// before the lookup, as every other entry point refuses it.  The first lookup
+// loads this file's device code on the device and so reserves the array there.
 moe_status scratch_address(void** out) {
     int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_UNSUPPORTED;
+    }
     if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess || major != 10) {
+        cudaGetLastError();
+        return MOE_ERR_UNSUPPORTED;
+    }
     std::lock_guard<std::mutex> lock(g_mu);
     if (!g_scratch_ptr[dev]) {
         void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();  // leave no sticky-looking error behind for the caller's next check
+            return MOE_ERR_CUDA;
+        }
         g_scratch_ptr[dev] = p;
     }
     *out = g_scratch_ptr[dev];

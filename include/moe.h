@@ -68,6 +68,7 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_E4M3 = 2 } moe_dtype;
 #define MOE_DEVERR_BAD_EXPERT 0x1u    /* a routed expert id outside [0, n_experts) */
 #define MOE_DEVERR_TIMEOUT    0x2u    /* a pipeline wait exceeded its limit */
 #define MOE_DEVERR_BAD_ROWS   0x4u    /* a schedule entry or a combine row's token outside its buffer */
+#define MOE_DEVERR_NONFINITE  0x8u    /* a router logit was NaN or infinite (a NaN ranks last) */
 
 /* Layer shape ("Teardown: DeepSeek-V3", At a glance + section 6; field guide
  * cutaway 02).  Constraints checked by every entry point:
@@ -406,8 +407,15 @@ MOE_API moe_status moe_ep_combine(int T, int d, int n_rows, const float* back_ro
  *   - If moe_workspace_size(cfg, T) exceeds MOE_NOALLOC_MAX_BYTES the call
  *     returns MOE_ERR_WORKSPACE and enqueues nothing; use moe_forward then.
  *   - The first call on a device looks up the array's device address for that
- *     device (cudaGetSymbolAddress, once per device, with the device current);
- *     make that first call before any stream capture.
+ *     device (cudaGetSymbolAddress, once per device, with the device current).
+ *     With CUDA's lazy module loading (the default since CUDA 12.2) that first
+ *     lookup is also what loads the library's device code on the device and
+ *     reserves the array, which goes through the driver's allocator and may
+ *     synchronise.  So make one warm-up call per device at initialisation,
+ *     before any stream capture and before the path that must not allocate;
+ *     later calls reserve nothing.
+ *   - A device that is not sm_100 returns MOE_ERR_UNSUPPORTED, as for every
+ *     other entry point.
  *   - Every call on a device shares the one array.  Calls whose work overlaps
  *     on the GPU (other streams, other host threads) race on it and give wrong
  *     results: order them on one stream or serialise them.  Whatever a

@@ -101,6 +101,14 @@ def test_no_device_means_unsupported_not_fallback(L):
     P = ctypes.c_void_p
     st = L.moe_permute(ctypes.byref(cfg), P(16), 4, P(16), P(16), P(16), P(16), None)
     assert st == moe.MOE_ERR_UNSUPPORTED
+    # the static-scratch forward refuses the same way, before it looks up its array
+    f = L.moe_forward_noalloc
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.POINTER(moe.MoeConfig), ctypes.POINTER(moe.MoeWeights), P, P, ctypes.c_int, P,
+                  ctypes.c_int, ctypes.c_int, P]
+    mw = moe.MoeWeights()
+    st = f(ctypes.byref(cfg), ctypes.byref(mw), P(16), P(16), 4, P(16), moe.MOE_BF16, 0, None)
+    assert st == moe.MOE_ERR_UNSUPPORTED
 
 
 def test_prenorm_and_block_arguments(L):

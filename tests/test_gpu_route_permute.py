@@ -59,6 +59,31 @@ def test_select_all_equal_logits():
     assert np.all(w == np.float32(0.125))
 
 
+def test_select_nonfinite_logits_are_flagged_and_ids_stay_valid():
+    """Logits must be finite (a precondition).  A NaN or infinite logit sets
+    MOE_DEVERR_NONFINITE; the NaN ranks last, so every token still gets k distinct
+    in-range ids, and tokens whose logits are finite route exactly as the oracle."""
+    wl = WORKLOADS["decode"]
+    T, E = 40, wl.n_experts
+    rng = np.random.default_rng(9)
+    l = (rng.standard_normal((T, E)) * 2).astype(np.float32)
+    l[3, :] = np.nan                                    # a whole token
+    l[5, :E // 2] = np.nan                              # half of the groups
+    l[7, 17] = np.nan
+    l[9, 40] = np.inf
+    b = np.zeros(E, np.float32)
+    assert moe.device_error() == 0
+    idx, w = _route(cfg_of(wl), None, None, torch.from_numpy(l).to(DEV), torch.from_numpy(b).to(DEV), T)
+    assert moe.device_error() & moe.MOE_DEVERR_NONFINITE
+    assert np.all((idx >= 0) & (idx < E))
+    assert all(len(set(r)) == wl.top_k for r in idx.tolist())
+    clean = [t for t in range(T) if np.all(np.isfinite(l[t]))]
+    ridx, rw = oracle.select(l[clean], b, wl.n_groups, wl.topk_groups, wl.top_k)
+    assert np.array_equal(idx[clean], ridx)
+    assert np.array_equal(w[clean].view(np.uint32), rw.view(np.uint32))
+    assert moe.device_error() == 0                      # read and cleared
+
+
 @pytest.mark.parametrize("name,T", [("tiny", 64), ("tiny", 129), ("decode", 128), ("decode", 300)])
 def test_router_logits_and_selection(name, T):
     wl = WORKLOADS[name]
