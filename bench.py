@@ -15,6 +15,11 @@ and of y out inside every step, through the C ABI's host-buffer entry point:
 `e2e.value` with the steps alternating between two streams (one step's copies
 overlap the other's kernels), `e2e.serial_value` one step after another.
 
+The default run (decode) adds, under "workloads", the metric's other
+configurations measured by the same code in the same process: prefill
+(T=4096), skewed routing (T=16384) and FP8 weights (T=8192), 20 steps each
+(--no-extra skips them).
+
 With N > 1 (launched by torchrun) every rank runs an independent replica of
 the layer on its own GPU and batch (weak scaling; the layer has no exchange
 step on one node without expert parallelism).  Rank 0 prints one JSON line.
@@ -38,16 +43,12 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
-# kernel per launch, from one ncu capture, keyed by workload; valid only while
-# the kernel sources hash to the recorded value.  profile_decode is captured
-# directly (the gate/up GEMM streams 30 routed + 1 shared expert weight sets);
-# decode is that capture scaled by weight sets streamed, 146 / 31 (traffic grows
-# with the touched experts: the profile_decode capture moves 0.99995 x its
-# algorithmic bytes).
-NCU_TRAFFIC = {
-    "profile_decode": (1_822_885_120, "7d5f411566a278e1"),
-    "decode": (8_585_200_888, "7d5f411566a278e1"),
-}
+# kernel per launch, from one ncu capture, keyed by workload: (bytes, kernel
+# source hash the capture was taken at, how the figure was obtained).  A figure
+# is reported only while the kernel sources still hash to the recorded value.
+NCU_TRAFFIC: dict = {}
+
+HBM_NOMINAL_GBS = 7700.0  # B200 (HGX) HBM3e nominal bandwidth, for context beside the measured copy peak
 
 
 def kernel_source_hash() -> str:
@@ -247,7 +248,9 @@ def roofline(F, B, seconds, peaks, peak_kind, fp8=False, sustained=False):
     if t_hbm >= t_tc:
         ach = B / seconds / 1e9
         return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(ach / peaks["hbm_gbs"], 4), "peak_source": peak_kind}
+                "frac": round(ach / peaks["hbm_gbs"], 4),
+                "peak_source": peak_kind + " copy bandwidth (read + write stream); a read-mostly kernel can exceed it",
+                "frac_of_nominal": round(ach / HBM_NOMINAL_GBS, 4), "nominal_gbs": HBM_NOMINAL_GBS}
     ach = F / seconds / 1e12
     src = peak_kind + (" sustained" if sustained else " burst") + (" bf16 x 2 (nominal e4m3/bf16 ratio)" if fp8 else "")
     out = {"bound": "tensor", "achieved": round(ach, 1), "peak": round(ptc, 1), "unit": "TFLOP/s",
@@ -258,19 +261,26 @@ def roofline(F, B, seconds, peaks, peak_kind, fp8=False, sustained=False):
 
 
 # --------------------------------------------------------------------------- oracle timing
-def _oracle_runner(wl, W, x, n_tokens):
-    """An oracle run on n_tokens of the batch (the CPU oracle alone; nothing of
-    the CUDA path).  The sampled tokens are chosen, among the first 64, to
-    share experts: that keeps the host copy of the weights small and leaves the
-    per-token cost unchanged (every token evaluates its routing plus k routed
-    experts and the shared expert).  Returns (run, n, threads)."""
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _oracle_runner(wl, W, x, n_tokens, threads):
+    """The CPU oracle alone (nothing of the CUDA path) on the batch.  Returns
+    (route, experts, n): route() runs the router GEMM (fp64), the selection and the
+    permutation on all T tokens; experts() runs the expert math and the combine on
+    n sampled tokens, chosen among the first 512 to share experts (that keeps the
+    host copy of the weights small; every token costs the same k routed + 1 shared
+    expert evaluations, so the per-token cost does not depend on the choice)."""
     import numpy as np
     import torch
 
     import oracle
 
     T = x.shape[0]
-    pool = min(T, 64)
 
     def u16(t):
         return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
@@ -278,18 +288,17 @@ def _oracle_runner(wl, W, x, n_tokens):
     def u8(t):
         return t.detach().contiguous().view(torch.uint8).cpu().numpy()
 
-    xp = x[:pool]
-    xp_h = xp.cpu().numpy() if xp.dtype == torch.float32 else u16(xp)
+    x_h = x.cpu().numpy() if x.dtype == torch.float32 else u16(x)
     wr_h = u16(W["w_router"])
     bias_h = W["bias"].cpu().numpy()
-    idx_h, _ = oracle.select(oracle.router_logits(xp_h, wr_h), bias_h, wl.n_groups, wl.topk_groups, wl.top_k)
+    pool = min(T, 512)
+    idx_p, _ = oracle.select(oracle.router_logits(x_h[:pool], wr_h), bias_h, wl.n_groups, wl.topk_groups, wl.top_k)
     chosen, experts = [], set()
     while len(chosen) < min(n_tokens, pool):
-        best = min((t for t in range(pool) if t not in chosen), key=lambda t: (len(set(idx_h[t]) - experts), t))
+        best = min((t for t in range(pool) if t not in chosen), key=lambda t: (len(set(idx_p[t]) - experts), t))
         chosen.append(best)
-        experts |= set(idx_h[best].tolist())
+        experts |= set(idx_p[best].tolist())
     toks = np.array(sorted(chosen), dtype=np.int32)
-    xs_h = xp_h[toks]
 
     conv = u8 if wl.fp8 else u16
     E = wl.n_experts
@@ -307,17 +316,34 @@ def _oracle_runner(wl, W, x, n_tokens):
                   ss_up=W["ss_up"].cpu().numpy(), ss_down=W["ss_down"].cpu().numpy())
     L = oracle.Layer(wl.d, E, wl.hidden, wl.shared_hidden, wl.top_k, wl.routed_scale, wg, wu, wd,
                      conv(W["ws_gate"]), conv(W["ws_up"]), conv(W["ws_down"]), x_is_f32=wl.x_f32, **kw)
-    threads = max(1, min(os.cpu_count() or 1, len(toks)))
+    routing = {}
 
-    def run():
-        # the oracle's whole path on the sampled tokens: router logits (fp64),
-        # selection, permutation, experts and combine
-        l = oracle.router_logits(xs_h, wr_h)
-        i2, w2 = oracle.select(l, bias_h, wl.n_groups, wl.topk_groups, wl.top_k)
-        oracle.permute(i2, wl.n_experts)
-        oracle.expert_tokens(L, xs_h, i2, w2, np.arange(len(toks)), n_threads=threads)
+    def route():
+        l = oracle.router_logits(x_h, wr_h)
+        routing["idx"], routing["w"] = oracle.select(l, bias_h, wl.n_groups, wl.topk_groups, wl.top_k)
+        oracle.permute(routing["idx"], wl.n_experts)
 
-    return run, len(toks), threads
+    def run_experts():
+        oracle.expert_tokens(L, x_h, routing["idx"], routing["w"], toks, n_threads=threads)
+
+    return route, run_experts, len(toks)
+
+
+def oracle_step_time(wl, route, run_experts, n):
+    """Seconds of one oracle step over the whole batch: routing and permutation of all
+    T tokens as timed, plus the sampled expert math scaled to T by its per-token cost."""
+    t0 = time.perf_counter()
+    route()
+    t1 = time.perf_counter()
+    run_experts()
+    t2 = time.perf_counter()
+    return (t1 - t0) + (t2 - t1) * wl.T / n, t1 - t0, t2 - t1
+
+
+def oracle_sample_desc(wl, n, threads):
+    return (f"router GEMM (fp64), selection and permutation on all {wl.T} tokens; expert math and combine on "
+            f"{n} of them (chosen to share experts) and scaled to {wl.T} by the per-token cost (every token costs "
+            f"k routed + 1 shared expert evaluations); fp64; {threads} host threads")
 
 
 def _cfg(wl):
@@ -344,8 +370,8 @@ def workload_desc(wl):
 
 # --------------------------------------------------------------------------- arms
 def run_reference(args, wl):
-    """The CPU oracle, as it stands, on the host cores: each step is a bounded
-    sample of the batch (see cpu_baseline.sample)."""
+    """The CPU oracle, as it stands, on the host cores: each step is the whole batch's
+    routing plus a bounded sample of its expert math (see cpu_baseline.sample)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
@@ -358,56 +384,73 @@ def run_reference(args, wl):
         return 0
     W = make_inputs(wl, dev)
     W = {k: v.to("cuda") for k, v in W.items()} if dev == "cuda" else W
-    n = args.cpu_sample or min(wl.T, 8)
-    run, n, threads = _oracle_runner(wl, W, W["x"], n)
+    threads = host_cores()
+    n = args.cpu_sample or min(wl.T, 2 * threads)
+    route, run_experts, n = _oracle_runner(wl, W, W["x"], n, threads)
     for _ in range(args.warmup):
-        run()
-    t0 = time.perf_counter()
+        oracle_step_time(wl, route, run_experts, n)
+    total = 0.0
     for _ in range(args.steps):
-        run()
-    dt = time.perf_counter() - t0
-    value = n * args.steps / dt
-    sample = (f"{n} of the {wl.T} tokens per step (tokens chosen to share experts; every token costs k routed + "
-              f"1 shared expert evaluations plus its routing)")
+        total += oracle_step_time(wl, route, run_experts, n)[0]
+    value = wl.T * args.steps / total
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": workload_desc(wl), "T": wl.T},
             "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
-                             "sample": sample},
+                             "sample": oracle_sample_desc(wl, n, threads)},
             "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
     return 0
 
 
-def run_ours(args, wl):
+class RunContext:
+    """One process per GPU: device, ranks, the barrier and the peaks."""
+
+    def __init__(self):
+        import torch
+        import torch.distributed as dist
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(self.local)
+        self.dev = torch.device("cuda", self.local)
+        if self.world > 1:
+            import datetime
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=self.dev)
+        self.peaks, self.peak_kind = load_peaks()
+
+    def barrier(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def close(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+def measure_layer(args, wl, steps, warmup, ctx, block=False):
+    """One workload of the layer (or of the pre-norm sublayer with block=True):
+    device-only steps, stage times, the end-to-end steps with host buffers, and the
+    accounting.  Every rank runs it (same collective steps in the same order);
+    returns (entry, W, x) with the timings already reduced as the max over ranks."""
     import torch
-    import torch.distributed as dist
 
     import fine_grained_moe_gemm_b200 as moe
     from workloads import make_inputs, make_norm_gain, make_stream
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    peaks, peak_kind = load_peaks()
+    dev, rank, world = ctx.dev, ctx.rank, ctx.world
+    peaks, peak_kind = ctx.peaks, ctx.peak_kind
     cfg = _cfg(wl)
     T = wl.T
     src_dev = "cpu" if wl.d <= 1024 else dev
     W = {k: v.to(dev) for k, v in make_inputs(wl, src_dev, seed=rank).items()}
     weights = {k: v for k, v in W.items() if k not in ("x", "bias")}
     x, bias = W["x"], W["bias"]
-    block = args.op == "block"
+    norm_g = None
     if block:  # the input is the residual stream h; the layer runs on RMSNorm(h) and adds h back
         x = W["x"] = make_stream(wl, dev, seed=rank)
         norm_g = W["norm_g"] = make_norm_gain(wl, dev, seed=rank)
@@ -422,21 +465,18 @@ def run_ours(args, wl):
         else:
             moe.moe_forward(cfg, weights, xin, bias, y, workspace=ws, stage_events=ev)
 
-    def step(ev=None):
-        forward(x, ev)
-
     # inputs smaller than twice the L2 would be served from it: write a buffer larger than
     # the L2 before every timed step and time the steps alone (events around each step)
     in_bytes = sum(v.numel() * v.element_size() for v in W.values())
     flush = torch.empty(4 * L2_BYTES, dtype=torch.uint8, device=dev) if in_bytes < 2 * L2_BYTES else None
 
-    for _ in range(max(args.warmup, 0)):
-        step()
+    for _ in range(max(warmup, 0)):
+        forward(x)
     torch.cuda.synchronize()
     if moe.device_error() != 0:
         raise RuntimeError("device error word set during warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     plan = moe.forward_plan(cfg, T)
     if block:
@@ -446,8 +486,8 @@ def run_ours(args, wl):
     # gaps); with an L2 flush between steps the steps are launched and timed one by one instead
     if not args.eager and flush is None:
         # stage times from eager steps (the graph runs the same kernels), then one captured step
-        for i in range(args.steps):
-            step(evs[i])
+        for i in range(steps):
+            forward(x, evs[i])
         torch.cuda.synchronize()
         cap = torch.cuda.Stream()
         cap.wait_stream(stream)
@@ -459,32 +499,34 @@ def run_ours(args, wl):
             raise RuntimeError("the captured step does not hold the planned kernels")
         graph.replay()
         torch.cuda.synchronize()
-    barrier()
+    ctx.barrier()
     torch.cuda.synchronize()
     n_launch0 = moe.launch_count()
-    with ClockSampler(local) as clk:
+    with ClockSampler(ctx.local) as clk:
         t_start.record(stream)
-        for i in range(args.steps):
+        for i in range(steps):
             if flush is not None:
                 flush.fill_(i & 0xff)
             if graph is not None:
                 graph.replay()
             else:
-                step(evs[i])
+                forward(x, evs[i])
         t_end.record(stream)
         torch.cuda.synchronize()
     # kernels that ran in the timed region: counted at launch, or the captured step's per replay
-    launches = moe.launch_count() - n_launch0 if graph is None else plan["launches"] * args.steps
-    if launches != plan["launches"] * args.steps:
+    launches = moe.launch_count() - n_launch0 if graph is None else plan["launches"] * steps
+    if launches != plan["launches"] * steps:
         raise RuntimeError(f"{launches} kernel launches in the timed region, the plan says "
                            f"{plan['launches']} per step")
-    barrier()
+    ctx.barrier()
     ms = t_start.elapsed_time(t_end) if flush is None else sum(e[0].elapsed_time(e[5]) for e in evs)
     stage_ms = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
                 for i, name in enumerate(moe.STAGES)}
     ms_max = max_over_ranks(ms, dev)
     if moe.device_error() != 0:
         raise RuntimeError("device error word set during the timed steps")
+    used_graph, flushed = graph is not None, flush is not None
+    del graph
 
     # end to end with host buffers: pinned x in, y out, every step.  The layer goes through
     # moe_forward_host (the C ABI call that takes host buffers and does the copies); the block,
@@ -493,7 +535,7 @@ def run_ours(args, wl):
     #   pipelined  steps alternate between two streams with two workspaces, so the copies of
     #              one step run on the copy engines while the other step's kernels run (the
     #              loop a server runs); timed from the first copy to the last one.
-    e2e_steps = max(1, args.steps)
+    e2e_steps = max(1, steps)
     x_host = x.cpu().pin_memory()
     y_hosts = [torch.empty((T, wl.d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     streams = [stream, torch.cuda.Stream()]
@@ -516,9 +558,10 @@ def run_ours(args, wl):
         else:
             moe.moe_forward_host(cfg, weights, x_host, bias, y_hosts[j], workspace=e2e_ws[j], stream=s)
 
-    e2e_serial_ms, e2e_pipe_ms = time_e2e(e2e_step, e2e_steps, args.warmup, streams, dev, barrier, flush)
+    e2e_serial_ms, e2e_pipe_ms = time_e2e(e2e_step, e2e_steps, warmup, streams, dev, ctx.barrier, flush)
     if moe.device_error() != 0:
         raise RuntimeError("device error word set during the end-to-end steps")
+    del e2e_ws, ws, flush
 
     # routed experts actually touched (for the byte accounting), through the ABI
     logits = torch.empty((T, wl.n_experts), dtype=torch.float32, device=dev)
@@ -537,70 +580,101 @@ def run_ours(args, wl):
     c = counts.cpu()
     U = int((c > 0).sum())
 
-    line = None
-    if rank == 0:
-        F, B = layer_accounting(wl, T, U, 2)
-        step_s = ms_max / args.steps / 1e3
-        k_name = max(("gate_up", "down+combine"), key=lambda n: stage_ms[n])
-        kF, kB = kernel_accounting(wl, T, U, "gate_up" if k_name == "gate_up" else "down")
-        sus = ms_max / 1e3 >= SUSTAINED_AFTER_S
-        kr = roofline(kF, kB, stage_ms[k_name] / 1e3, peaks, peak_kind, fp8=wl.fp8, sustained=sus)
-        tr = NCU_TRAFFIC.get(wl.name)
-        kr["traffic"] = tr[0] if tr and tr[1] == kernel_source_hash() else None
-        kr["kernel"] = ("moe_gemm2" if plan["cta_pair"] else "moe_gemm") + ("_fp8" if plan["fp8"] else "") + \
-            "_kernel<" + ("GATEUP" if k_name == "gate_up" else "DOWN") + ", BN=" + str(plan["token_tile"]) + ">"
-        lr = roofline(F, B, step_s, peaks, peak_kind, fp8=wl.fp8, sustained=sus)
-        # the router GEMM stays bf16 in the FP8 layer
-        F_router = 2 * T * wl.n_experts * wl.d
-        t_tc = ((F - F_router) / (tensor_peak(peaks, wl.fp8, sus) * 1e12)
-                + F_router / (tensor_peak(peaks, False, sus) * 1e12))
-        t_roof = max(t_tc, B / (peaks["hbm_gbs"] * 1e9))
-        lr["roofline_ms"] = round(t_roof * 1e3, 4)
-        lr["frac_of_roofline_time"] = round(t_roof / step_s, 4)
-        lr["algorithmic_bytes"] = B
-        lr["algorithmic_flops"] = F
-        kr["algorithmic_bytes"] = kB
-        kr["algorithmic_flops"] = kF
-        value = world * T * args.steps / (ms_max / 1e3)
-        line = {
-            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if wl.fp8 else "bf16",
-            "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights; no checkpoint)",
-            "config": {"workload": ("MoE sublayer y = h + MoE(RMSNorm(h)), eps 1e-6, bf16 residual stream; "
-                                    if block else "") + workload_desc(wl), "T": T, "experts_touched": U,
-                       "max_rows_per_expert": int(c.max()), "mean_rows_per_touched_expert": round(T * wl.top_k / U, 1),
-                       "l2": ("inputs larger than L2: the touched expert weights "
-                              f"({(U + 1) * 3 * wl.hidden * wl.d * (1 if wl.fp8 else 2) / 1e9:.2f} GB) stream from HBM "
-                              "every step") if flush is None else
-                             ("L2 flushed before every timed step (a 504 MiB buffer written between steps, outside "
-                              "the per-step CUDA events that are summed)"),
-                       "parallelism": f"replicas x{world} (no data-path collective)",
-                       "launch": "CUDA-graph replay of the captured step" if graph is not None else "eager"},
-            "roofline": kr,
-            "layer_roofline": lr,
-            "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
-            "e2e": e2e_entry(world * T * e2e_steps, e2e_serial_ms, e2e_pipe_ms, x.numel() * x.element_size(),
-                             y.numel() * y.element_size(),
-                             "moe_forward_block + copies" if block else "moe_forward_host (host buffers)"),
-            "gpu_launches": launches,
-            "plan": plan,
-            "clocks": clk.summary(),
-            "kernel_source": kernel_source_hash(),
-        }
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-    if rank == 0:
-        if world == 1 and not args.no_cpu_baseline:
-            n = args.cpu_sample or min(T, 8)
-            run, n, threads = _oracle_runner(wl, W, x, n)
-            t0 = time.perf_counter()
-            run()
-            dt = time.perf_counter() - t0
-            line["cpu_baseline"] = {"value": round(n / dt, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
-                                    "sample": f"{n} of the {T} tokens (chosen to share experts; every token costs "
-                                              "its routing plus k routed + 1 shared expert evaluations), fp64"}
+    F, B = layer_accounting(wl, T, U, 2)
+    step_s = ms_max / steps / 1e3
+    k_name = max(("gate_up", "down+combine"), key=lambda n: stage_ms[n])
+    kF, kB = kernel_accounting(wl, T, U, "gate_up" if k_name == "gate_up" else "down")
+    sus = ms_max / 1e3 >= SUSTAINED_AFTER_S
+    kr = roofline(kF, kB, stage_ms[k_name] / 1e3, peaks, peak_kind, fp8=wl.fp8, sustained=sus)
+    kr["kernel"] = ("moe_gemm2" if plan["cta_pair"] else "moe_gemm") + ("_fp8" if plan["fp8"] else "") + \
+        "_kernel<" + ("GATEUP" if k_name == "gate_up" else "DOWN") + ", BN=" + str(plan["token_tile"]) + ">"
+    tr = NCU_TRAFFIC.get(wl.name + (":block" if block else ""))
+    ok = tr is not None and tr[1] == kernel_source_hash()
+    kr["traffic"] = tr[0] if ok else None
+    kr["traffic_source"] = tr[2] if ok else "none: no ncu capture of the current kernel sources for this workload"
+    lr = roofline(F, B, step_s, peaks, peak_kind, fp8=wl.fp8, sustained=sus)
+    # the router GEMM stays bf16 in the FP8 layer
+    F_router = 2 * T * wl.n_experts * wl.d
+    t_tc = ((F - F_router) / (tensor_peak(peaks, wl.fp8, sus) * 1e12)
+            + F_router / (tensor_peak(peaks, False, sus) * 1e12))
+    t_roof = max(t_tc, B / (peaks["hbm_gbs"] * 1e9))
+    lr["roofline_ms"] = round(t_roof * 1e3, 4)
+    lr["frac_of_roofline_time"] = round(t_roof / step_s, 4)
+    lr["algorithmic_bytes"] = B
+    lr["algorithmic_flops"] = F
+    kr["algorithmic_bytes"] = kB
+    kr["algorithmic_flops"] = kF
+    value = world * T * steps / (ms_max / 1e3)
+    entry = {
+        "value": round(value, 1), "unit": UNIT, "steps": steps, "warmup": warmup,
+        "ms_per_step": round(ms_max / steps, 4), "dtype": "e4m3" if wl.fp8 else "bf16",
+        "config": {"workload": ("MoE sublayer y = h + MoE(RMSNorm(h)), eps 1e-6, bf16 residual stream; "
+                                if block else "") + workload_desc(wl), "T": T, "experts_touched": U,
+                   "max_rows_per_expert": int(c.max()), "mean_rows_per_touched_expert": round(T * wl.top_k / U, 1),
+                   "l2": ("inputs larger than L2: the touched expert weights "
+                          f"({(U + 1) * 3 * wl.hidden * wl.d * (1 if wl.fp8 else 2) / 1e9:.2f} GB) stream from HBM "
+                          "every step") if not flushed else
+                         ("L2 flushed before every timed step (a 504 MiB buffer written between steps, outside "
+                          "the per-step CUDA events that are summed)"),
+                   "parallelism": f"replicas x{world} (no data-path collective)",
+                   "launch": "CUDA-graph replay of the captured step" if used_graph else "eager"},
+        "roofline": kr,
+        "layer_roofline": lr,
+        "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+        "e2e": e2e_entry(world * T * e2e_steps, e2e_serial_ms, e2e_pipe_ms, x.numel() * x.element_size(),
+                         y.numel() * y.element_size(),
+                         "moe_forward_block + copies" if block else "moe_forward_host (host buffers)"),
+        "gpu_launches": launches,
+        "plan": plan,
+        "clocks": clk.summary(),
+    }
+    return entry, W, x
+
+
+EXTRA_WORKLOADS = ("prefill", "skewed", "fp8")
+EXTRA_STEPS = 20
+
+
+def run_ours(args, wl):
+    import torch
+
+    from workloads import WORKLOADS
+
+    ctx = RunContext()
+    block = args.op == "block"
+    entry, W, x = measure_layer(args, wl, args.steps, args.warmup, ctx, block=block)
+    cpu = None
+    if ctx.rank == 0 and ctx.world == 1 and not args.no_cpu_baseline and not block:
+        threads = host_cores()
+        n = args.cpu_sample or min(wl.T, 2 * threads)
+        route, run_experts, n = _oracle_runner(wl, W, x, n, threads)
+        sec, t_route, t_exp = oracle_step_time(wl, route, run_experts, n)
+        cpu = {"value": round(wl.T / sec, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": oracle_sample_desc(wl, n, threads),
+               "seconds": {"routing_all_tokens": round(t_route, 3), "experts_sample": round(t_exp, 3)}}
+    del W, x
+    torch.cuda.empty_cache()
+    # the metric's other configurations, measured by the same code in the same run
+    subs = {}
+    if not args.no_extra and not block and args.tokens == 0 and wl.name == "decode":
+        for name in EXTRA_WORKLOADS:
+            e, W2, x2 = measure_layer(args, WORKLOADS[name], min(args.steps, EXTRA_STEPS), args.warmup, ctx)
+            del W2, x2
+            torch.cuda.empty_cache()
+            subs[name] = e
+    ctx.close()
+    if ctx.rank == 0:
+        line = {"metric": METRIC, "value": entry["value"], "unit": UNIT, "n_gpus": ctx.world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": entry["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": entry["dtype"],
+                "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights; no checkpoint)"}
+        for k in ("config", "roofline", "layer_roofline", "stages_ms", "e2e", "gpu_launches", "plan", "clocks"):
+            line[k] = entry[k]
+        if subs:
+            line["workloads"] = subs
+        line["kernel_source"] = kernel_source_hash()
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
         print(json.dumps(line))
     return 0
 
@@ -745,8 +819,11 @@ def main():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
-    p.add_argument("--cpu-sample", type=int, default=0, help="tokens of the oracle sample (0: min(T, 8))")
+    p.add_argument("--cpu-sample", type=int, default=0,
+                   help="tokens of the oracle's expert-math sample (0: min(T, 2 x host cores))")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-extra", action="store_true",
+                   help="decode only: skip the prefill, skewed and fp8 lines added under 'workloads'")
     p.add_argument("--tokens", type=int, default=0, help="override the workload's T (sweeps; default: as named)")
     p.add_argument("--eager", action="store_true",
                    help="launch every timed step from the host instead of replaying the captured step as a CUDA "

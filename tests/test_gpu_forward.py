@@ -75,11 +75,20 @@ def forward_routing(wl, W, x):
     return ridx, rw
 
 
-def oracle_y(wl, W, x, tokens):
+def oracle_y(wl, W, x, tokens, chunk=16):
+    """The oracle's output for the listed tokens, routed as the forward routed.  The
+    tokens go in chunks, each with a host copy of only the experts it uses, so the
+    host memory stays bounded however many tokens are checked."""
     idx, w = forward_routing(wl, W, x)
-    need = np.unique(idx[tokens])
-    L = oracle_layer(wl, W, need)
-    return oracle.expert_tokens(L, x_host(x), idx, w, tokens)
+    xh = x_host(x)
+    out = []
+    tokens = np.asarray(tokens, dtype=np.int32)
+    for c0 in range(0, tokens.size, chunk):
+        part = tokens[c0:c0 + chunk]
+        L = oracle_layer(wl, W, np.unique(idx[part]))
+        out.append(oracle.expert_tokens(L, xh, idx, w, part))
+        del L
+    return np.concatenate(out) if out else np.zeros((0, wl.d))
 
 
 # ----------------------------------------------------------------------------- tiny workload (full check)
@@ -117,12 +126,35 @@ def _sample(T, n, seed=0):
     return np.array(sorted(s), dtype=np.int32)
 
 
-@pytest.mark.parametrize("T", [128, 1, 37])
+def _spread(T, n, seed=0):
+    """n tokens spread over the batch: one from each of n equal slices (so every token
+    chunk of the GEMMs' schedules is hit), plus the first and the last."""
+    rng = np.random.default_rng(seed)
+    edges = np.linspace(0, T, n + 1).astype(np.int64)
+    s = {0, T - 1} | {int(rng.integers(a, b)) for a, b in zip(edges[:-1], edges[1:]) if b > a}
+    return np.array(sorted(s), dtype=np.int32)
+
+
+def test_decode_every_token():
+    """The benchmarked decode batch (T = 128): every token, every feature, fp32 and bf16
+    outputs, against the oracle."""
+    wl = WORKLOADS["decode"]
+    W = inputs("decode", "cuda")
+    x = W["x"]
+    toks = np.arange(wl.T, dtype=np.int32)
+    ref = oracle_y(wl, W, x, toks)
+    y = run_forward(wl, W, x, torch.float32)
+    assert_close_rms(y.cpu().numpy(), ref, REL)
+    yb = run_forward(wl, W, x, torch.bfloat16)
+    assert_close_bf16(yb, ref, REL)
+
+
+@pytest.mark.parametrize("T", [1, 37])
 def test_decode(T):
     wl = WORKLOADS["decode"]
     W = inputs("decode", "cuda")
     x = make_x(wl, "cuda", T=T) if T != wl.T else W["x"]
-    toks = _sample(T, 6)
+    toks = np.arange(T, dtype=np.int32)
     ref = oracle_y(wl, W, x, toks)
     y = run_forward(wl, W, x, torch.float32)
     assert_close_rms(y.cpu().numpy()[toks], ref, REL)
@@ -137,7 +169,7 @@ def test_mid_batches_sampled(T):
     wl = WORKLOADS["prefill"]
     W = inputs("prefill", "cuda")
     x = make_x(wl, "cuda", T=T)
-    toks = _sample(T, 4, seed=T)
+    toks = _spread(T, 8, seed=T)
     ref = oracle_y(wl, W, x, toks)
     yb = run_forward(wl, W, x, torch.bfloat16)
     assert_close_bf16(yb[torch.from_numpy(toks).long().to(DEV)], ref, REL)
@@ -149,7 +181,7 @@ def test_prefill_sampled():
     wl = WORKLOADS["prefill"]
     W = inputs("prefill", "cuda")
     x = W["x"]
-    toks = _sample(wl.T, 6, seed=1)
+    toks = _spread(wl.T, 32, seed=1)
     ref = oracle_y(wl, W, x, toks)
     yb = run_forward(wl, W, x, torch.bfloat16)
     assert_close_bf16(yb[torch.from_numpy(toks).long().to(DEV)], ref, REL)
@@ -163,7 +195,7 @@ def test_large_batch_sampled():
     W = inputs("prefill", "cuda")
     T = 65536
     x = make_x(wl, "cuda", T=T)
-    toks = _sample(T, 3, seed=3)
+    toks = _spread(T, 16, seed=3)
     ref = oracle_y(wl, W, x, toks)
     yb = run_forward(wl, W, x, torch.bfloat16)
     assert_close_bf16(yb[torch.from_numpy(toks).long().to(DEV)], ref, REL)
@@ -173,7 +205,7 @@ def test_skewed_sampled():
     wl = WORKLOADS["skewed"]
     W = inputs("skewed", "cuda")
     x = W["x"]
-    toks = _sample(wl.T, 4, seed=2)
+    toks = _spread(wl.T, 32, seed=2)
     ref = oracle_y(wl, W, x, toks)
     y = run_forward(wl, W, x, torch.float32)
     assert_close_rms(y.cpu().numpy()[toks], ref, REL)
