@@ -21,12 +21,14 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+DEBUG_LIB_PATH = os.path.join(_HERE, "libmoe_b200_debug.so")
 _DEFAULT_LIB_PATH = LIB_PATH
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "moe.h")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_DEVICE, MOE_ERR_CUDA = range(6)
 MOE_F32, MOE_BF16, MOE_E4M3 = 0, 1, 2
-MOE_DEVERR_BAD_EXPERT, MOE_DEVERR_TIMEOUT, MOE_DEVERR_BAD_ROWS, MOE_DEVERR_NONFINITE = 1, 2, 4, 8
+MOE_DEVERR_BAD_EXPERT, MOE_DEVERR_TIMEOUT, MOE_DEVERR_BAD_ROWS, MOE_DEVERR_NONFINITE, MOE_DEVERR_BOUNDS = 1, 2, 4, 8, 16
+MOE_DEBUG_TABLE_ROW_TOK, MOE_DEBUG_TABLE_ROW_OFF = 0, 1
 
 _lib = None
 _lock = threading.Lock()
@@ -56,6 +58,72 @@ class MoeWeights(ctypes.Structure):
         "ws_gate", "ws_up", "ws_down", "ss_gate", "ss_up", "ss_down")]
 
 
+def _configure(L):
+    """Result and argument types of every entry point of a loaded library."""
+    P, I = ctypes.c_void_p, ctypes.c_int
+    L.moe_workspace_size.restype = ctypes.c_size_t
+    L.moe_workspace_size.argtypes = [ctypes.POINTER(MoeConfig), I]
+    L.moe_route.restype = I
+    L.moe_route.argtypes = [ctypes.POINTER(MoeConfig), P, P, P, P, I, P, P, P]
+    L.moe_permute.restype = I
+    L.moe_permute.argtypes = [ctypes.POINTER(MoeConfig), P, I, P, P, P, P, P]
+    L.moe_forward.restype = I
+    L.moe_forward.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, I, P, I, I, P,
+                              ctypes.c_size_t, P]
+    L.moe_forward_ex.restype = I
+    L.moe_forward_ex.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, I, P, I, I, P,
+                                 ctypes.c_size_t, P, P, P]
+    L.moe_host_workspace_size.restype = ctypes.c_size_t
+    L.moe_host_workspace_size.argtypes = [ctypes.POINTER(MoeConfig), I, I]
+    L.moe_forward_host.restype = I
+    L.moe_forward_host.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, I, P, I, I, P,
+                                   ctypes.c_size_t, P]
+    L.moe_ep_max_send_rows.restype = I
+    L.moe_ep_max_send_rows.argtypes = [ctypes.POINTER(MoeConfig), I, I]
+    L.moe_ep_dispatch.restype = I
+    L.moe_ep_dispatch.argtypes = [ctypes.POINTER(MoeConfig), I, P, P, P, I, P, P, P, P, P, P, P]
+    L.moe_experts_routed_workspace_size.restype = ctypes.c_size_t
+    L.moe_experts_routed_workspace_size.argtypes = [ctypes.POINTER(MoeConfig), I, I]
+    L.moe_experts_routed.restype = I
+    L.moe_experts_routed.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), I, I, P, I, P, P,
+                                     P, P, ctypes.c_size_t, P]
+    L.moe_ep_combine.restype = I
+    L.moe_ep_combine.argtypes = [I, I, I, P, P, P, P, P, P]
+    L.moe_rmsnorm.restype = I
+    L.moe_rmsnorm.argtypes = [P, P, ctypes.c_float, I, I, P, P, P, P]
+    L.moe_block_workspace_size.restype = ctypes.c_size_t
+    L.moe_block_workspace_size.argtypes = [ctypes.POINTER(MoeConfig), I]
+    L.moe_forward_block.restype = I
+    L.moe_forward_block.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, ctypes.c_float,
+                                    P, P, I, P, P, ctypes.c_size_t, P, P, P]
+    L.moe_dense_workspace_size.restype = ctypes.c_size_t
+    L.moe_dense_workspace_size.argtypes = [I, I, I, I, I]
+    L.moe_dense_ffn.restype = I
+    L.moe_dense_ffn.argtypes = [I, I, I, I, P, P, P, P, P, P, P, I, P, I, I, P, ctypes.c_size_t, P, P]
+    L.moe_forward_plan.restype = I
+    L.moe_forward_plan.argtypes = [ctypes.POINTER(MoeConfig), I, I, ctypes.c_void_p]
+    L.moe_selftest_wait_timeout.restype = I
+    L.moe_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, P]
+    L.moe_launch_count.restype = ctypes.c_ulonglong
+    L.moe_launch_count.argtypes = []
+    L.moe_update_bias.restype = I
+    L.moe_update_bias.argtypes = [ctypes.POINTER(MoeConfig), P, P, ctypes.c_float, P]
+    L.moe_quantize_act.restype = I
+    L.moe_quantize_act.argtypes = [P, I, I, P, P, P]
+    L.moe_device_error.restype = I
+    L.moe_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), P]
+    L.moe_status_string.restype = ctypes.c_char_p
+    L.moe_status_string.argtypes = [I]
+    L.moe_abi_version.restype = I
+    L.moe_forward_noalloc.restype = I
+    L.moe_forward_noalloc.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, I, P, I, I, P]
+    L.moe_debug_build.restype = I
+    L.moe_debug_build.argtypes = []
+    L.moe_debug_corrupt_next.restype = I
+    L.moe_debug_corrupt_next.argtypes = [I, I, I]
+    return L
+
+
 def lib():
     """The loaded ``libmoe_b200.so``.  The in-tree library is (re)built first when it is
     missing or older than its sources and nvcc is at hand; without it the call raises
@@ -73,64 +141,26 @@ def lib():
             if not os.path.exists(LIB_PATH):
                 raise RuntimeError(f"{LIB_PATH} is missing: build it with fine_grained_moe_gemm_b200.build.build() "
                                    "(there is no CPU fallback)")
-            L = ctypes.CDLL(LIB_PATH)
-            P, I = ctypes.c_void_p, ctypes.c_int
-            L.moe_workspace_size.restype = ctypes.c_size_t
-            L.moe_workspace_size.argtypes = [ctypes.POINTER(MoeConfig), I]
-            L.moe_route.restype = I
-            L.moe_route.argtypes = [ctypes.POINTER(MoeConfig), P, P, P, P, I, P, P, P]
-            L.moe_permute.restype = I
-            L.moe_permute.argtypes = [ctypes.POINTER(MoeConfig), P, I, P, P, P, P, P]
-            L.moe_forward.restype = I
-            L.moe_forward.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, I, P, I, I, P,
-                                      ctypes.c_size_t, P]
-            L.moe_forward_ex.restype = I
-            L.moe_forward_ex.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, I, P, I, I, P,
-                                         ctypes.c_size_t, P, P, P]
-            L.moe_host_workspace_size.restype = ctypes.c_size_t
-            L.moe_host_workspace_size.argtypes = [ctypes.POINTER(MoeConfig), I, I]
-            L.moe_forward_host.restype = I
-            L.moe_forward_host.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, I, P, I, I, P,
-                                           ctypes.c_size_t, P]
-            L.moe_ep_max_send_rows.restype = I
-            L.moe_ep_max_send_rows.argtypes = [ctypes.POINTER(MoeConfig), I, I]
-            L.moe_ep_dispatch.restype = I
-            L.moe_ep_dispatch.argtypes = [ctypes.POINTER(MoeConfig), I, P, P, P, I, P, P, P, P, P, P, P]
-            L.moe_experts_routed_workspace_size.restype = ctypes.c_size_t
-            L.moe_experts_routed_workspace_size.argtypes = [ctypes.POINTER(MoeConfig), I, I]
-            L.moe_experts_routed.restype = I
-            L.moe_experts_routed.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), I, I, P, I, P, P,
-                                             P, P, ctypes.c_size_t, P]
-            L.moe_ep_combine.restype = I
-            L.moe_ep_combine.argtypes = [I, I, I, P, P, P, P, P, P]
-            L.moe_rmsnorm.restype = I
-            L.moe_rmsnorm.argtypes = [P, P, ctypes.c_float, I, I, P, P, P, P]
-            L.moe_block_workspace_size.restype = ctypes.c_size_t
-            L.moe_block_workspace_size.argtypes = [ctypes.POINTER(MoeConfig), I]
-            L.moe_forward_block.restype = I
-            L.moe_forward_block.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, ctypes.c_float,
-                                            P, P, I, P, P, ctypes.c_size_t, P, P, P]
-            L.moe_dense_workspace_size.restype = ctypes.c_size_t
-            L.moe_dense_workspace_size.argtypes = [I, I, I, I, I]
-            L.moe_dense_ffn.restype = I
-            L.moe_dense_ffn.argtypes = [I, I, I, I, P, P, P, P, P, P, P, I, P, I, I, P, ctypes.c_size_t, P, P]
-            L.moe_forward_plan.restype = I
-            L.moe_forward_plan.argtypes = [ctypes.POINTER(MoeConfig), I, I, ctypes.c_void_p]
-            L.moe_selftest_wait_timeout.restype = I
-            L.moe_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, P]
-            L.moe_launch_count.restype = ctypes.c_ulonglong
-            L.moe_launch_count.argtypes = []
-            L.moe_update_bias.restype = I
-            L.moe_update_bias.argtypes = [ctypes.POINTER(MoeConfig), P, P, ctypes.c_float, P]
-            L.moe_quantize_act.restype = I
-            L.moe_quantize_act.argtypes = [P, I, I, P, P, P]
-            L.moe_device_error.restype = I
-            L.moe_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), P]
-            L.moe_status_string.restype = ctypes.c_char_p
-            L.moe_status_string.argtypes = [I]
-            L.moe_abi_version.restype = I
-            _lib = L
+            _lib = _configure(ctypes.CDLL(LIB_PATH))
     return _lib
+
+
+_debug_lib = None
+
+
+def debug_lib():
+    """The checking build ``libmoe_b200_debug.so`` (the same entry points; kernels
+    check every table-dependent access against its buffer and flag
+    MOE_DEVERR_BOUNDS instead of touching memory outside it).  Built with the
+    regular library."""
+    global _debug_lib
+    lib()  # builds both libraries when they are stale
+    with _lock:
+        if _debug_lib is None:
+            if not os.path.exists(DEBUG_LIB_PATH):
+                raise RuntimeError(f"{DEBUG_LIB_PATH} is missing: build it with fine_grained_moe_gemm_b200.build.build()")
+            _debug_lib = _configure(ctypes.CDLL(DEBUG_LIB_PATH))
+    return _debug_lib
 
 
 def declared_symbols() -> list[str]:

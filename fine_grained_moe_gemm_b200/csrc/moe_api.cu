@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 #include <string.h>
 
@@ -10,6 +11,20 @@
 
 #include "../../include/moe.h"
 #include "moe_launch.h"
+
+#ifdef MOE_DEBUG
+constexpr bool kDebugBuild = true;   // the checking build (libmoe_b200_debug.so)
+#else
+constexpr bool kDebugBuild = false;
+#endif
+
+// Checking build: the one-shot table corruption armed by moe_debug_corrupt_next
+// (tests of the bounds checks).  The regular build never arms it.
+struct DebugCorruption {
+    int table = -1, index = 0, value = 0;
+};
+static std::mutex g_debug_mu;
+static DebugCorruption g_debug_corruption;
 
 using namespace moe;
 
@@ -219,6 +234,36 @@ Workspace layout(const moe_config* c, int T, void* base) {
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+// NVTX ranges around the host-side enqueue of each stage (names "moe.<stage>"),
+// nested in one range per entry point: a profiler's timeline groups the kernels
+// by stage, and ncu can select them with --nvtx-include.  Header-only NVTX: with
+// no tool attached each push/pop is a call through a null stub.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
+// Consecutive stages of one call: next() closes the open stage range, if any,
+// and opens the named one; the destructor closes the last.
+class NvtxStages {
+    bool open_ = false;
+
+public:
+    NvtxStages() = default;
+    NvtxStages(const NvtxStages&) = delete;
+    NvtxStages& operator=(const NvtxStages&) = delete;
+    void next(const char* name) {
+        if (open_) nvtxRangePop();
+        nvtxRangePushA(name);
+        open_ = true;
+    }
+    ~NvtxStages() {
+        if (open_) nvtxRangePop();
+    }
+};
+
 // The kernels one forward call runs, decided from the shapes and the SM count.
 struct Plan {
     int bn;              // token rows per grouped-GEMM tile
@@ -350,6 +395,19 @@ extern "C" {
 
 int moe_abi_version(void) { return MOE_ABI_VERSION; }
 
+int moe_debug_build(void) { return kDebugBuild ? 1 : 0; }
+
+moe_status moe_debug_corrupt_next(int table, int index, int value) {
+    if (table != -1 && table != MOE_DEBUG_TABLE_ROW_TOK && table != MOE_DEBUG_TABLE_ROW_OFF)
+        return MOE_ERR_INVALID_ARG;
+    if (!kDebugBuild) return MOE_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> g(g_debug_mu);
+    g_debug_corruption.table = table;
+    g_debug_corruption.index = index;
+    g_debug_corruption.value = value;
+    return MOE_OK;
+}
+
 const char* moe_status_string(moe_status s) {
     switch (s) {
         case MOE_OK: return "MOE_OK";
@@ -369,6 +427,7 @@ size_t moe_workspace_size(const moe_config* cfg, int T_max) {
 
 moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router, float* logits, const float* bias,
                      int T, int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
+    NvtxRange nvtx_call("moe_route");
     moe_status st = check_config(cfg);
     if (st != MOE_OK) return st;
     if (T < 0) return MOE_ERR_INVALID_ARG;
@@ -432,6 +491,7 @@ moe_status moe_update_bias(const moe_config* cfg, const int32_t* counts, float* 
 
 moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, int T, int32_t* counts, int32_t* offsets,
                        int32_t* src, int32_t* inv, moe_stream_t stream) {
+    NvtxRange nvtx_call("moe_permute");
     moe_status st = check_config(cfg);
     if (st != MOE_OK) return st;
     if (T < 0) return MOE_ERR_INVALID_ARG;
@@ -462,6 +522,7 @@ moe_status moe_forward(const moe_config* cfg, const moe_weights* wt, const void*
 moe_status moe_forward_ex(const moe_config* cfg, const moe_weights* wt, const void* x, const float* bias, int T,
                           void* y, moe_dtype y_dtype, int accumulate, void* workspace, size_t ws_bytes,
                           moe_stream_t stream, const moe_stage_events* events, const moe_routing_out* routing) {
+    NvtxRange nvtx_call("moe_forward");
     return forward_impl(cfg, wt, x, bias, T, y, y_dtype, accumulate, workspace, ws_bytes, stream, events, routing,
                         nullptr, 0.0f);
 }
@@ -521,6 +582,7 @@ moe_status moe_dense_ffn(int d, int hidden, moe_dtype act_dtype, moe_dtype weigh
                          const void* w_up, const void* w_down, const float* s_gate, const float* s_up,
                          const float* s_down, const void* x, int T, void* y, moe_dtype y_dtype, int accumulate,
                          void* workspace, size_t ws_bytes, moe_stream_t stream, const moe_stage_events* events) {
+    NvtxRange nvtx_call("moe_dense_ffn");
     if (!dense_shape_ok(d, hidden, act_dtype, weight_dtype)) {
         const bool bad_shape = d <= 0 || hidden <= 0 || d % 128 || hidden % 128;
         return bad_shape ? MOE_ERR_INVALID_ARG : MOE_ERR_UNSUPPORTED;
@@ -576,6 +638,7 @@ moe_status moe_dense_ffn(int d, int hidden, moe_dtype act_dtype, moe_dtype weigh
 moe_status moe_forward_block(const moe_config* cfg, const moe_weights* wt, const void* norm_g, float eps,
                              const void* h, const float* bias, int T, void* y, void* workspace, size_t ws_bytes,
                              moe_stream_t stream, const moe_stage_events* events, const moe_routing_out* routing) {
+    NvtxRange nvtx_call("moe_forward_block");
     moe_status st = check_config(cfg);
     if (st != MOE_OK) return st;
     if (cfg->act_dtype != MOE_BF16 || cfg->d > 8 * NORM_MAX_VEC * NORM_THREADS) return MOE_ERR_UNSUPPORTED;
@@ -597,6 +660,7 @@ size_t moe_host_workspace_size(const moe_config* cfg, int T_max, moe_dtype y_dty
 moe_status moe_forward_host(const moe_config* cfg, const moe_weights* wt, const void* x_host, const float* bias,
                             int T, void* y_host, moe_dtype y_dtype, int accumulate, void* workspace, size_t ws_bytes,
                             moe_stream_t stream) {
+    NvtxRange nvtx_call("moe_forward_host");
     moe_status st = check_config(cfg);
     if (st != MOE_OK) return st;
     if (T < 0 || (y_dtype != MOE_F32 && y_dtype != MOE_BF16)) return MOE_ERR_INVALID_ARG;
@@ -749,18 +813,21 @@ moe_status run_experts(const moe_config* cfg, const moe_weights* wt, const Works
     // one group of all T rows in token order (the dense FFN) with bf16 x: the token
     // operand is x itself, no gathered copy
     const bool direct_b = E == 0 && !fp8 && cfg->act_dtype == MOE_BF16;
+    NvtxStages nv;
+    nv.next(fp8 ? "moe.quantize+gather" : "moe.gather");
     if (fp8) {
         if ((!act_quantised && launch_quant_act(static_cast<const __nv_bfloat16*>(x), T, d, W.x_q, W.sx, s) != cudaSuccess) ||
-            launch_gather_fp8(W.x_q, W.sx, d, W.row_tok, W.row_off + NG, rows_max, W.xq_perm, W.sxT, di.sm_count,
+            launch_gather_fp8(W.x_q, W.sx, d, T, W.row_tok, W.row_off + NG, rows_max, W.xq_perm, W.sxT, di.sm_count,
                               s) != cudaSuccess)
             return MOE_ERR_CUDA;
-    } else if (!direct_b && launch_gather(x, cfg->act_dtype == MOE_F32, d, W.row_tok, W.row_off + NG, rows_max,
+    } else if (!direct_b && launch_gather(x, cfg->act_dtype == MOE_F32, d, T, W.row_tok, W.row_off + NG, rows_max,
                                           W.x_perm, di.sm_count, s) != cudaSuccess) {
         return MOE_ERR_CUDA;
     }
     mark(2);
 
     // (4) gate/up grouped GEMM with the SwiGLU epilogue -> h_perm
+    nv.next("moe.gate_up");
     auto wmap = [&](CUtensorMap* m, const void* p, uint64_t rows, uint64_t cols, uint32_t box_rows) {
         return fp8 ? map_u8(m, p, rows, cols, box_rows) : map_bf16(m, p, rows, cols, box_rows);
     };
@@ -786,6 +853,7 @@ moe_status run_experts(const moe_config* cfg, const moe_weights* wt, const Works
         return MOE_ERR_CUDA;
     g.item_off = W.item_gu;
     g.row_off = W.row_off;
+    g.rows_cap = rows_max;
     g.n_groups = NG;
     g.n_routed = E;
     g.K_routed = g.K_shared = d;
@@ -815,6 +883,7 @@ moe_status run_experts(const moe_config* cfg, const moe_weights* wt, const Works
     mark(3);
 
     // (5) down GEMM, routing-weight scale and un-permute scatter into fp32
+    nv.next("moe.down+combine");
     float* yacc = y_dtype == MOE_F32 ? static_cast<float*>(y) : W.y_acc;
     if ((y_dtype == MOE_BF16 || !accumulate) &&
         cudaMemsetAsync(yacc, 0, (size_t)T * d * sizeof(float), s) != cudaSuccess)
@@ -834,6 +903,8 @@ moe_status run_experts(const moe_config* cfg, const moe_weights* wt, const Works
         return MOE_ERR_CUDA;
     dn.item_off = W.item_dn;
     dn.row_off = W.row_off;
+    dn.rows_cap = rows_max;
+    dn.y_rows = T;
     dn.n_groups = NG;
     dn.n_routed = E;
     dn.K_routed = H;
@@ -859,12 +930,36 @@ moe_status run_experts(const moe_config* cfg, const moe_weights* wt, const Works
     if (edn != cudaSuccess) return MOE_ERR_CUDA;
     mark(4);
 
+    nv.next("moe.cast");
     if (y_dtype == MOE_BF16 &&
         launch_finalize_bf16(W.y_acc, static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(y),
                              (size_t)T * d, s) != cudaSuccess)
         return MOE_ERR_CUDA;
     mark(5);
     return MOE_OK;
+}
+
+// Applies (and disarms) an armed corruption to this call's tables, on the stream,
+// after the permutation has written them.  An index outside the table does nothing.
+cudaError_t apply_debug_corruption(const Workspace& W, int rows_max, int n_groups, cudaStream_t s) {
+    if (!kDebugBuild) return cudaSuccess;
+    DebugCorruption c;
+    {
+        std::lock_guard<std::mutex> g(g_debug_mu);
+        c = g_debug_corruption;
+        g_debug_corruption.table = -1;
+    }
+    int32_t* base = nullptr;
+    int n = 0;
+    if (c.table == MOE_DEBUG_TABLE_ROW_TOK) {
+        base = W.row_tok;
+        n = rows_max;
+    } else if (c.table == MOE_DEBUG_TABLE_ROW_OFF) {
+        base = W.row_off;
+        n = n_groups + 1;
+    }
+    if (!base || c.index < 0 || c.index >= n) return cudaSuccess;
+    return launch_debug_poke(base + c.index, c.value, s);
 }
 
 moe_status forward_impl(const moe_config* cfg, const moe_weights* wt, const void* x, const float* bias, int T,
@@ -907,11 +1002,13 @@ moe_status forward_impl(const moe_config* cfg, const moe_weights* wt, const void
     auto mark = [&](int i) {
         if (events && events->ev[i]) cudaEventRecord((cudaEvent_t)events->ev[i], s);
     };
+    NvtxStages nv;
     // (0) pre-norm of the sublayer: the layer runs on x = RMSNorm(h) and adds h back at
     //     the end; in the FP8 layer the same pass writes the activation codes and scales
     mark(0);
     const void* residual = accumulate ? y : nullptr;
     if (norm_g) {
+        nv.next("moe.rmsnorm");
         __nv_bfloat16* xhat = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(workspace) + W.bytes);
         if (launch_rmsnorm(static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(norm_g), T, d,
                            eps, xhat, fp8 ? W.x_q : nullptr, fp8 ? W.sx : nullptr, s) != cudaSuccess)
@@ -920,11 +1017,13 @@ moe_status forward_impl(const moe_config* cfg, const moe_weights* wt, const void
         x = xhat;
     }
     // (1)+(2) router and selection
+    nv.next("moe.route");
     st = route_impl(cfg, di, x, wt->w_router, W.logits, bias, T, W.idx, W.w, s, W.part, plan.router_parts);
     if (st != MOE_OK) return st;
     mark(1);
 
     // (3) permutation + tile schedules
+    nv.next("moe.permute");
     PermuteArgs pa;
     memset(&pa, 0, sizeof(pa));
     pa.idx = W.idx;
@@ -949,6 +1048,7 @@ moe_status forward_impl(const moe_config* cfg, const moe_weights* wt, const void
     pa.mt_dn = pair ? d / 512 : (d + 255) / 256;  // pair8: 256 down rows per item, as the 1-CTA kernels
     const cudaError_t ep = plan.permute_multi ? launch_permute_multi(pa, W.hist, s) : launch_permute(pa, s);
     if (ep != cudaSuccess) return MOE_ERR_CUDA;
+    if (apply_debug_corruption(W, T * k + cfg->n_shared * T, E + cfg->n_shared, s) != cudaSuccess) return MOE_ERR_CUDA;
     return run_experts(cfg, wt, W, plan, di, T, x, norm_g != nullptr, y, y_dtype, accumulate, residual, s, events, 1);
 }
 

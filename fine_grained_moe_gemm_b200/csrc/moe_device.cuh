@@ -19,6 +19,25 @@ __device__ unsigned int g_dev_error = 0;
 
 __device__ __forceinline__ void set_dev_error(unsigned int bits) { atomicOr(&g_dev_error, bits); }
 
+// The checking build (compiled with MOE_DEBUG): table-dependent accesses are
+// checked against their buffers first.  dbg_ok(ok) is true in the regular
+// build (the check folds away); in the checking build a false `ok` sets
+// MOE_DEVERR_BOUNDS and returns false, and the caller skips the access or
+// replaces it with an in-bounds one.
+#ifdef MOE_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+
+__device__ __forceinline__ bool dbg_ok(bool ok) {
+    if (kDebugChecks && !ok) {
+        set_dev_error(MOE_DEVERR_BOUNDS);
+        return false;
+    }
+    return true;
+}
+
 // ---------------------------------------------------------------- sigmoid_spec
 // The router's sigmoid (the llm-vis "MoE router" box: logits.sigmoid()), pinned
 // to a fixed sequence of correctly rounded fp32 operations so that the CPU

@@ -108,6 +108,8 @@ __device__ __forceinline__ Item decode_item(const GemmArgs& P, int i) {
     int local = i - __ldg(&P.item_off[lo]);
     int r0 = __ldg(&P.row_off[lo]);
     int ng = __ldg(&P.row_off[lo + 1]) - r0;
+    // checking build: a group that owns items has rows (else the chunk count below is 0)
+    if (kDebugChecks && P.rows_cap > 0 && !dbg_ok(ng > 0)) ng = 1;
     int nch = (ng + BN - 1) / BN;
     const int ms = local / nch;  // tile-major, split, then token chunk (chunks of a weight slice run together)
     it.m = ms / it.n_splits;
@@ -117,6 +119,16 @@ __device__ __forceinline__ Item decode_item(const GemmArgs& P, int i) {
     it.nvalid = min(BN, ng - c * BN);
     it.shared = lo >= P.n_routed;
     it.K = it.shared ? P.K_shared : P.K_routed;
+    if (kDebugChecks && P.rows_cap > 0) {
+        // checking build: the item's rows inside the permuted buffers and its weight
+        // tile inside the expert (every role decodes the same replacement)
+        const int mt = it.shared ? P.mt_shared : P.mt_routed;
+        if (!dbg_ok(it.row0 >= 0 && it.nvalid >= 1 && it.row0 + it.nvalid <= P.rows_cap && it.m >= 0 && it.m < mt)) {
+            it.row0 = 0;
+            it.nvalid = min(BN, P.rows_cap);
+            it.m = 0;
+        }
+    }
     return it;
 }
 
@@ -297,6 +309,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) moe_gemm_kernel(const __grid_
                 if (MODE == GEMM_DOWN && c0 + lane < it.nvalid) {
                     cf_l = __ldg(&P.row_coef[it.row0 + c0 + lane]);
                     tok_l = __ldg(&P.row_tok[it.row0 + c0 + lane]);
+                    // checking build: the token's y row exists (else the row is skipped)
+                    if (kDebugChecks && !dbg_ok((unsigned)tok_l < (unsigned)P.y_rows)) tok_l = -1;
                 }
                 tmem_ld32x2(t0 + (uint32_t)c0, t1 + (uint32_t)c0, v0, v1);
                 if (MODE == GEMM_GATEUP) {
@@ -313,7 +327,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) moe_gemm_kernel(const __grid_
                     for (int jj = 0; jj < 32; ++jj) {
                         const float cf = __shfl_sync(0xffffffffu, cf_l, jj);
                         const int tok = __shfl_sync(0xffffffffu, tok_l, jj);
-                        if (c0 + jj < it.nvalid) {
+                        if (c0 + jj < it.nvalid && (!kDebugChecks || tok >= 0)) {
                             float* yr = P.y + (size_t)tok * P.ldy;
                             if (ok0) atomicAdd(yr + f0, v0[jj] * cf);
                             if (ok1) atomicAdd(yr + f1, v1[jj] * cf);

@@ -296,6 +296,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
                 if (MODE == GEMM_DOWN && c0 + lane < it.nvalid) {
                     cf_l = __ldg(&P.row_coef[it.row0 + c0 + lane]);
                     tok_l = __ldg(&P.row_tok[it.row0 + c0 + lane]);
+                    // checking build: the token's y row exists (else the row is skipped)
+                    if (kDebugChecks && !dbg_ok((unsigned)tok_l < (unsigned)P.y_rows)) tok_l = -1;
                 }
                 tmem_ld32x2(t0 + (uint32_t)c0, t1 + (uint32_t)c0, v0, v1);
                 if (MODE == GEMM_GATEUP) {
@@ -312,7 +314,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
                     for (int jj = 0; jj < 32; ++jj) {
                         const float cf = __shfl_sync(0xffffffffu, cf_l, jj);
                         const int tok = __shfl_sync(0xffffffffu, tok_l, jj);
-                        if (c0 + jj < it.nvalid) {
+                        if (c0 + jj < it.nvalid && (!kDebugChecks || tok >= 0)) {
                             float* yr = P.y + (size_t)tok * P.ldy;
                             if (ok0) atomicAdd(yr + f0, v0[jj] * cf);
                             if (ok1) atomicAdd(yr + f1, v1[jj] * cf);

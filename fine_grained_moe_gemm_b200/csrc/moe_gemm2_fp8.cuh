@@ -401,12 +401,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
                         // this lane's permuted row, handed to the other lanes by shuffles
                         const bool okr = c0 + lane < it.nvalid;
                         const float cf_l = okr ? __ldg(&P.row_coef[it.row0 + c0 + lane]) : 0.0f;
-                        const int tok_l = okr ? __ldg(&P.row_tok[it.row0 + c0 + lane]) : 0;
+                        int tok_l = okr ? __ldg(&P.row_tok[it.row0 + c0 + lane]) : 0;
+                        // checking build: the token's y row exists (else the row is skipped)
+                        if (kDebugChecks && okr && !dbg_ok((unsigned)tok_l < (unsigned)P.y_rows)) tok_l = -1;
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
                             const float cf = __shfl_sync(0xffffffffu, cf_l, j);
                             const int tok = __shfl_sync(0xffffffffu, tok_l, j);
-                            if (c0 + j < it.nvalid) {
+                            if (c0 + j < it.nvalid && (!kDebugChecks || tok >= 0)) {
                                 float* yr = P.y + (size_t)tok * P.ldy;
                                 if (okf) atomicAdd(yr + f, acc[c][j] * cf);
                             }

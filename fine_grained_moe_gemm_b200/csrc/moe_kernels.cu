@@ -468,14 +468,17 @@ __global__ void __launch_bounds__(PERM_TB) permute_scatter_kernel(PermuteArgs a,
 }
 
 // ============================================================================ gather
-__global__ void __launch_bounds__(256) gather_rows_kernel(const void* __restrict__ x, int x_f32, int d,
+__global__ void __launch_bounds__(256) gather_rows_kernel(const void* __restrict__ x, int x_f32, int d, int n_tok,
                                                           const int32_t* __restrict__ row_tok,
-                                                          const int32_t* __restrict__ n_rows_dev,
+                                                          const int32_t* __restrict__ n_rows_dev, int rows_cap,
                                                           __nv_bfloat16* __restrict__ xp) {
-    const int n_rows = *n_rows_dev;
+    int n_rows = *n_rows_dev;
+    // checking build: the row count fits the permuted buffer, every row's token exists
+    if (kDebugChecks && !dbg_ok(n_rows >= 0 && n_rows <= rows_cap)) n_rows = n_rows < 0 ? 0 : rows_cap;
     const int nvec = d / 8;  // 8 bf16 per 16-byte vector
     for (int r = blockIdx.x; r < n_rows; r += gridDim.x) {
         const int t = row_tok[r];
+        if (kDebugChecks && !dbg_ok((unsigned)t < (unsigned)n_tok)) continue;  // uniform over the block
         uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)r * d);
         if (x_f32) {
             const float4* srcf = reinterpret_cast<const float4*>(static_cast<const float*>(x) + (size_t)t * d);
@@ -520,13 +523,16 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const __nv_bfloat16* __r
 }
 
 __global__ void __launch_bounds__(256) gather_fp8_kernel(const uint8_t* __restrict__ xq, const float* __restrict__ sx,
-                                                         int d, const int32_t* __restrict__ row_tok,
+                                                         int d, int n_tok, const int32_t* __restrict__ row_tok,
                                                          const int32_t* __restrict__ n_rows_dev, int rows_ld,
                                                          uint8_t* __restrict__ xpq, float* __restrict__ sxT) {
-    const int n_rows = *n_rows_dev;
+    int n_rows = *n_rows_dev;
+    // checking build: the row count fits the permuted buffers, every row's token exists
+    if (kDebugChecks && !dbg_ok(n_rows >= 0 && n_rows <= rows_ld)) n_rows = n_rows < 0 ? 0 : rows_ld;
     const int nvec = d / 16, nb = d / 128;
     for (int r = blockIdx.x; r < n_rows; r += gridDim.x) {
         const int t = row_tok[r];
+        if (kDebugChecks && !dbg_ok((unsigned)t < (unsigned)n_tok)) continue;  // uniform over the block
         const uint4* src = reinterpret_cast<const uint4*>(xq + (size_t)t * d);
         uint4* dst = reinterpret_cast<uint4*>(xpq + (size_t)r * d);
         for (int v = threadIdx.x; v < nvec; v += blockDim.x) dst[v] = src[v];
@@ -970,13 +976,13 @@ cudaError_t launch_quant_act(const __nv_bfloat16* x, int T, int d, uint8_t* q, f
     return cudaGetLastError();
 }
 
-cudaError_t launch_gather_fp8(const uint8_t* xq, const float* sx, int d, const int32_t* row_tok,
+cudaError_t launch_gather_fp8(const uint8_t* xq, const float* sx, int d, int n_tok, const int32_t* row_tok,
                               const int32_t* n_rows_dev, int max_rows, uint8_t* xpq, float* sxT, int n_sm,
                               cudaStream_t s) {
     int grid = max_rows < n_sm * 8 ? max_rows : n_sm * 8;
     if (grid < 1) grid = 1;
     note_launch();
-    gather_fp8_kernel<<<grid, 256, 0, s>>>(xq, sx, d, row_tok, n_rows_dev, max_rows, xpq, sxT);
+    gather_fp8_kernel<<<grid, 256, 0, s>>>(xq, sx, d, n_tok, row_tok, n_rows_dev, max_rows, xpq, sxT);
     return cudaGetLastError();
 }
 
@@ -1053,12 +1059,20 @@ cudaError_t launch_permute_multi(const PermuteArgs& a, int32_t* hist, cudaStream
     return cudaGetLastError();
 }
 
-cudaError_t launch_gather(const void* x, bool x_f32, int d, const int32_t* row_tok, const int32_t* n_rows_dev,
+cudaError_t launch_gather(const void* x, bool x_f32, int d, int n_tok, const int32_t* row_tok, const int32_t* n_rows_dev,
                           int max_rows, __nv_bfloat16* x_perm, int n_sm, cudaStream_t s) {
     int grid = max_rows < n_sm * 8 ? max_rows : n_sm * 8;
     if (grid < 1) grid = 1;
     note_launch();
-    gather_rows_kernel<<<grid, 256, 0, s>>>(x, x_f32 ? 1 : 0, d, row_tok, n_rows_dev, x_perm);
+    gather_rows_kernel<<<grid, 256, 0, s>>>(x, x_f32 ? 1 : 0, d, n_tok, row_tok, n_rows_dev, max_rows, x_perm);
+    return cudaGetLastError();
+}
+
+__global__ void debug_poke_kernel(int32_t* p, int v) { *p = v; }
+
+cudaError_t launch_debug_poke(int32_t* p, int v, cudaStream_t s) {
+    note_launch();
+    debug_poke_kernel<<<1, 1, 0, s>>>(p, v);
     return cudaGetLastError();
 }
 
@@ -1126,7 +1140,7 @@ cudaError_t launch_ep_dispatch(const int32_t* idx, const float* w, int T, int k,
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || T == 0) return e;
     const int max_rows = T * (k < R ? k : R);
-    if ((e = launch_gather(x, x_f32, d, send_tok, offsets + R, max_rows, send_x, n_sm, s)) != cudaSuccess) return e;
+    if ((e = launch_gather(x, x_f32, d, T, send_tok, offsets + R, max_rows, send_x, n_sm, s)) != cudaSuccess) return e;
     int grid = (max_rows * k + 255) / 256;
     grid = grid < n_sm * 4 ? grid : n_sm * 4;
     note_launch();

@@ -45,6 +45,9 @@ struct GemmArgs {
     uint8_t* hq;               // GATEUP FP8 output codes [rows, ldh]
     float* hsT;                // GATEUP FP8 output scales [ldh/128][hs_ld]
     int hs_ld;
+    // checking build: rows of the B / h buffers (0: items are not checked) and of y
+    int rows_cap;
+    int y_rows;
 };
 
 enum { MODE_GATEUP = 0, MODE_DOWN = 1, MODE_LOGITS = 2 };
@@ -98,14 +101,17 @@ cudaError_t launch_ep_dispatch(const int32_t* idx, const float* w, int T, int k,
 cudaError_t launch_ep_combine(const float* back, const int32_t* send_tok, int n_rows, int T, int d, float* acc,
                               int n_sm, cudaStream_t s);
 // x_perm[r, :] = x[row_tok[r], :] (fp32 input rounded to bf16) for r < row_off[n_groups]
-cudaError_t launch_gather(const void* x, bool x_f32, int d, const int32_t* row_tok, const int32_t* n_rows_dev,
-                          int max_rows, __nv_bfloat16* x_perm, int n_sm, cudaStream_t s);
+// (checking build: row_tok entries against n_tok, the row count against max_rows)
+cudaError_t launch_gather(const void* x, bool x_f32, int d, int n_tok, const int32_t* row_tok,
+                          const int32_t* n_rows_dev, int max_rows, __nv_bfloat16* x_perm, int n_sm, cudaStream_t s);
 // q[t, :], sx[t, b]: per-token, per-128-channel e4m3 quantisation of bf16 x
 cudaError_t launch_quant_act(const __nv_bfloat16* x, int T, int d, uint8_t* q, float* sx, cudaStream_t s);
 // xpq[r, :] = xq[row_tok[r], :]; sxT[b][r] = sx[row_tok[r], b] for r < row_off[n_groups]
-cudaError_t launch_gather_fp8(const uint8_t* xq, const float* sx, int d, const int32_t* row_tok,
+cudaError_t launch_gather_fp8(const uint8_t* xq, const float* sx, int d, int n_tok, const int32_t* row_tok,
                               const int32_t* n_rows_dev, int max_rows, uint8_t* xpq, float* sxT, int n_sm,
                               cudaStream_t s);
+// checking build, tests only: *p = v on the stream
+cudaError_t launch_debug_poke(int32_t* p, int v, cudaStream_t s);
 int gemm_fp8_smem_bytes(int mode, int bn);
 // CTA-pair (2-SM MMA) bf16 grouped GEMM, 256 token rows per item; grid even.
 cudaError_t launch_gemm2(int mode, const GemmArgs* args, int grid, cudaStream_t s);

@@ -69,6 +69,9 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_E4M3 = 2 } moe_dtype;
 #define MOE_DEVERR_TIMEOUT    0x2u    /* a pipeline wait exceeded its limit */
 #define MOE_DEVERR_BAD_ROWS   0x4u    /* a schedule entry or a combine row's token outside its buffer */
 #define MOE_DEVERR_NONFINITE  0x8u    /* a router logit was NaN or infinite (a NaN ranks last) */
+#define MOE_DEVERR_BOUNDS     0x10u   /* checking build only: a table entry, row range or TMA
+                                         coordinate outside its buffer (the access was skipped
+                                         or replaced by an in-bounds one) */
 
 /* Layer shape ("Teardown: DeepSeek-V3", At a glance + section 6; field guide
  * cutaway 02).  Constraints checked by every entry point:
@@ -436,6 +439,34 @@ MOE_API const char* moe_status_string(moe_status s);
 
 /* MOE_ABI_VERSION of the loaded library. */
 MOE_API int moe_abi_version(void);
+
+/* ---- Checking build ------------------------------------------------------
+ * The library also comes as libmoe_b200_debug.so, the same sources compiled
+ * with MOE_DEBUG.  Its kernels check, before every access that depends on a
+ * device-built table, that the access stays inside its buffer: the token of
+ * each permuted row (x rows when gathering, y rows in the combine), the row
+ * count and the row range of every grouped-GEMM work item against the
+ * permuted buffers, and each item's weight tile against the expert's weight
+ * matrix (so every TMA coordinate lies inside its tensor map).  A failed
+ * check sets MOE_DEVERR_BOUNDS and skips the access, or replaces the work
+ * item with an in-bounds one whose output is discarded as wrong; nothing
+ * traps.  It stands in for a memory checker, at the cost of a few
+ * instructions per table read.  The pages have no counterpart: this is
+ * build tooling around the layer. */
+
+/* 1 in the checking build, 0 in the regular one. */
+MOE_API int moe_debug_build(void);
+
+#define MOE_DEBUG_TABLE_ROW_TOK 0   /* token of permuted row `index`: [n_rows] int32 */
+#define MOE_DEBUG_TABLE_ROW_OFF 1   /* first permuted row of group `index`: [groups + 1] int32 */
+
+/* Checking build only, for tests of the checks: arms a one-shot change of the
+ * next moe_forward / moe_forward_ex call (in any thread), which after its
+ * permutation writes `value` into entry `index` of the named device table,
+ * as a corrupted table would hold it.  An index outside the table leaves it
+ * unchanged.  table = -1 disarms.  Returns MOE_ERR_UNSUPPORTED in the regular
+ * build and MOE_ERR_INVALID_ARG for an unknown table; touches no device. */
+MOE_API moe_status moe_debug_corrupt_next(int table, int index, int value);
 
 #ifdef __cplusplus
 }
