@@ -133,7 +133,7 @@ int pick_bn(long long rows_per_expert) {
 constexpr int kBoxRows = 32;  // token rows per B-operand TMA box
 constexpr int kFp8MaxBn = 64;  // FP8 GEMMs hold their promoted sums in registers
 constexpr int kPermuteMultiMinT = 1024;  // tokens above which the permutation runs on many CTAs
-constexpr int kPairBoxRows = 16;  // token rows per B box in the CTA-pair GEMM (each CTA loads half)
+constexpr int kPairBoxRows = 64;  // token rows per B box in the CTA-pair GEMMs (PAIR_BOX_ROWS)
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 

@@ -28,7 +28,11 @@
 namespace moe {
 
 constexpr int PAIR_BN = 256;       // token rows per item (whole pair)
-constexpr int PAIR_BOX_ROWS = 16;  // token rows per B TMA box (each CTA loads N/2 rows)
+// Token rows per B TMA box (each CTA loads N/2 rows, rounded up to whole boxes;
+// rows past the item's own are loaded and ignored).  Wide boxes: one TMA
+// instruction costs a few hundred cycles of the issuing thread whatever its
+// size, so a stage is loaded in as few instructions as its tiles allow.
+constexpr int PAIR_BOX_ROWS = 64;
 // Sixteen epilogue warps (four per TMEM lane quarter): the accumulators are
 // single-buffered, so the MMA of the next item waits for the epilogue to drain
 // them, and four warps per SM sub-partition drain them about twice as fast as
@@ -41,6 +45,7 @@ struct Gemm2Cfg {
     static constexpr int A_TILE = 128 * 128;
     static constexpr int A_BYTES = 2 * A_TILE;              // this CTA's slices of the two tiles
     static constexpr int B_BYTES = PAIR_BN / 2 * 128;       // this CTA's half of the token rows
+    static_assert(B_BYTES % (PAIR_BOX_ROWS * 128) == 0, "B tile holds whole boxes");
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int MISC_BYTES = 1024;
     static constexpr int STAGES = (227 * 1024 - 1024 - MISC_BYTES) / STAGE_BYTES > 6
@@ -193,8 +198,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
                 const int KB = it.K / 64;
                 int n_mma = (it.nvalid + 31) & ~31;
                 const int nh = n_mma / 2;                          // this CTA's token rows
-                const int nbox = nh / PAIR_BOX_ROWS;
-                const uint32_t bytes = 2u * (uint32_t)(C::A_BYTES + nh * 128);
+                const int nbox = (nh + PAIR_BOX_ROWS - 1) / PAIR_BOX_ROWS;
+                const uint32_t bytes = 2u * (uint32_t)(C::A_BYTES + nbox * PAIR_BOX_ROWS * 128);
                 const CUtensorMap* m0;
                 const CUtensorMap* m1;
                 int r0, r1;

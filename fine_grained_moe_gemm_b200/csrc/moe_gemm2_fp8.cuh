@@ -26,14 +26,25 @@
 namespace moe {
 
 constexpr int PAIR8_BN = 128;  // token rows per item (whole pair)
+// Warps 0, 2, 3: TMA producers; warp 1: TMEM allocator and MMA issuer; warps 4-11:
+// eight promotion warps, two per TMEM lane quarter, each promoting 64 of the 128
+// token columns.  (Sixteen warps of 32 columns read TMEM faster but ran the layer
+// 15-25 % slower: per-block overheads doubled and registers dropped to 96.)
+constexpr int PAIR8_EPI_WARPS = 8;
+constexpr int PAIR8_NGRP = PAIR8_EPI_WARPS / 4;            // column groups
+constexpr int PAIR8_NCH = PAIR8_BN / (32 * PAIR8_NGRP);    // 32-column chunks per warp
+constexpr int PAIR8_EPI_BEGIN = 4;
+constexpr int PAIR8_THREADS = 32 * (PAIR8_EPI_BEGIN + PAIR8_EPI_WARPS);
+static_assert((PAIR8_NCH == 1 || PAIR8_NCH == 2) && PAIR8_NGRP * PAIR8_NCH * 32 == PAIR8_BN, "column split");
 
 struct Gemm2Fp8Cfg {
     static constexpr int A_BYTES = 128 * 128;                 // 128 rows x 128 e4m3
     static constexpr int B_BYTES = PAIR8_BN / 2 * 128;        // this CTA's 64 token rows
+    static_assert(B_BYTES % (PAIR_BOX_ROWS * 128) == 0, "B tile holds whole boxes");
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;     // 24 KB
     static constexpr int STAGES = 7;
-    static constexpr int XUP_STRIDE = 65;                     // padded [feature][column] fp32
-    static constexpr int XUP_BYTES = 2 * 64 * XUP_STRIDE * 4; // up sums handed to the gate warps
+    static constexpr int XUP_STRIDE = PAIR8_NCH * 32 + 1;     // padded [feature][column] fp32
+    static constexpr int XUP_BYTES = PAIR8_NGRP * 64 * XUP_STRIDE * 4;  // up sums handed to the gate warps
     static constexpr int MISC_BYTES = 6144;
     static constexpr int NUM_P = 4;                           // TMEM partial buffers
     static constexpr int P_COLS = PAIR8_BN;
@@ -85,7 +96,7 @@ __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_
 }
 
 template <int MODE>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR8_THREADS, 1)
     moe_gemm2_fp8_kernel(const __grid_constant__ GemmArgs P) {
     using C = Gemm2Fp8Cfg;
     extern __shared__ uint8_t smem_raw[];
@@ -98,15 +109,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     uint64_t* empty = full + C::STAGES;          // both: stage consumed
     uint64_t* pfull = empty + C::STAGES;         // both: partial written
     uint64_t* pempty = pfull + C::NUM_P;         // leader: partial promoted by both CTAs
-    uint64_t* xbar = pempty + C::NUM_P;          // both: [2 parity][2 groups] peer's column maxima arrived
-    uint64_t* drain = xbar + 4;
+    uint64_t* xbar = pempty + C::NUM_P;          // both: [2 parity][groups] peer's column maxima arrived
+    uint64_t* drain = xbar + 2 * PAIR8_NGRP;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    volatile int* warp_ok = reinterpret_cast<volatile int*>(tmem_slot + 2);  // [8]
-    float* sc_rows = reinterpret_cast<float*>(misc + 512);    // [8 warps][64]   scales of a K block
-    float* cmax = reinterpret_cast<float*>(misc + 2560);      // [2 groups][2 chunks][2 warps][32] column maxima
-    float* xmax = reinterpret_cast<float*>(misc + 3584);      // [2 parity][2 groups][64] peer's column maxima
-    float* sinv = reinterpret_cast<float*>(misc + 4608);      // [2 groups][64] inverse scales
+    volatile int* warp_ok = reinterpret_cast<volatile int*>(tmem_slot + 2);  // [epilogue warps]
+    constexpr int GCOLS = PAIR8_NCH * 32;                     // columns of one warp
+    float* sc_rows = reinterpret_cast<float*>(misc + 512);    // [epilogue warps][GCOLS] scales of a K block
+    float* cmax = reinterpret_cast<float*>(misc + 2560);      // [groups][chunks][2 gate warps][32] column maxima
+    float* xmax = reinterpret_cast<float*>(misc + 3584);      // [2 parity][groups][GCOLS] peer's column maxima
+    float* sinv = reinterpret_cast<float*>(misc + 4608);      // [groups][GCOLS] inverse scales
+    static_assert(PAIR8_EPI_WARPS * GCOLS * 4 <= 2048 && PAIR8_NGRP * GCOLS * 2 * 4 <= 1024 &&
+                      2 * PAIR8_NGRP * GCOLS * 4 <= 1024 && PAIR8_NGRP * GCOLS * 4 <= 1024,
+                  "misc layout");
+    static_assert((2 * C::STAGES + 2 * C::NUM_P + 2 * PAIR8_NGRP + 1) * 8 + 8 + 4 * PAIR8_EPI_WARPS <= 512,
+                  "barriers and flags");
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -115,14 +132,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], MODE == GEMM_GATEUP ? 3 : 2);  // the leader's producers of the stage
             mbar_init(&empty[s], 1);
         }
         for (int a = 0; a < C::NUM_P; ++a) {
             mbar_init(&pfull[a], 1);
-            mbar_init(&pempty[a], 2 * GEMM_EPI_THREADS / 32);
+            mbar_init(&pempty[a], 2 * PAIR8_EPI_WARPS);
         }
-        for (int a = 0; a < 4; ++a) mbar_init(&xbar[a], 1);  // the peer's q0 warp of the group arrives
+        for (int a = 0; a < 2 * PAIR8_NGRP; ++a) mbar_init(&xbar[a], 1);  // the peer's q0 warp of the group arrives
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -147,9 +164,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     const int cluster_id = blockIdx.x >> 1;
     const int n_clusters = gridDim.x >> 1;
 
-    if (warp == 0) {
-        if (lane == 0) {
-            // ------------------------------------------------ TMA producer (both CTAs)
+    if (warp == 0 || warp == 2 || warp == 3) {
+        // ------------------------------------------------ TMA producers (both CTAs)
+        // Three issuing warps, each with its own share of every stage: warp 0 the
+        // gate rows (GATEUP) or the whole weight tile (DOWN), warp 2 the up rows
+        // (GATEUP), warp 3 the token rows.  One thread issues a TMA instruction
+        // every few hundred cycles whatever its size, so one thread per operand.
+        const int role = warp == 0 ? 0 : warp - 1;  // 0 A/gate, 1 up, 2 B
+        if (lane == 0 && !(MODE == GEMM_DOWN && role == 1)) {
             const uint64_t pol_w = l2_policy_evict_first();
             const uint64_t pol_x = l2_policy_evict_last();
             const uint32_t full0 = mapa_shared(smem_u32(&full[0]), 0);
@@ -159,8 +181,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
                 const Item it = decode_item<PAIR8_BN>(P, i);
                 const int KB = it.K / 128;
                 const int nh = ((it.nvalid + 31) & ~31) / 2;
-                const int nbox = nh / PAIR_BOX_ROWS;
-                const uint32_t bytes = 2u * (uint32_t)(C::A_BYTES + nh * 128);
+                const int nbox = (nh + PAIR_BOX_ROWS - 1) / PAIR_BOX_ROWS;
+                // bytes this role brings into the stage, both CTAs together
+                const uint32_t bytes = role == 2 ? 2u * (uint32_t)(nbox * PAIR_BOX_ROWS * 128)
+                                       : MODE == GEMM_GATEUP ? 2u * 64u * 128u : 2u * (uint32_t)C::A_BYTES;
                 const int base = it.shared ? 0 : it.g * P.rows_per_expert;
                 const int brow = it.row0 + (int)rank * nh;
                 bool ok = true;
@@ -170,18 +194,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
                     uint8_t* sb = sa + C::A_BYTES;
                     const uint32_t fb = full0 + (uint32_t)(stage * 8);
                     if (leader) mbar_arrive_expect_tx(&full[stage], bytes);
-                    if (MODE == GEMM_GATEUP) {
+                    if (role == 2) {
+                        for (int bx = 0; bx < nbox; ++bx)
+                            tma_load_2d_pair(sb + bx * PAIR_BOX_ROWS * 128, &P.b, kb * 128, brow + bx * PAIR_BOX_ROWS,
+                                             fb, pol_x);
+                    } else if (MODE == GEMM_GATEUP) {
                         // 64 gate rows over 64 up rows of this CTA's 64 features
                         const int r = base + it.m * 128 + (int)rank * 64;
-                        tma_load_2d_pair(sa, it.shared ? &P.s0 : &P.a0, kb * 128, r, fb, pol_w);
-                        tma_load_2d_pair(sa + 64 * 128, it.shared ? &P.s1 : &P.a1, kb * 128, r, fb, pol_w);
+                        if (role == 0) tma_load_2d_pair(sa, it.shared ? &P.s0 : &P.a0, kb * 128, r, fb, pol_w);
+                        else tma_load_2d_pair(sa + 64 * 128, it.shared ? &P.s1 : &P.a1, kb * 128, r, fb, pol_w);
                     } else {
                         tma_load_2d_pair(sa, it.shared ? &P.s0 : &P.a0, kb * 128, base + it.m * 256 + (int)rank * 128,
                                          fb, pol_w);
                     }
-                    for (int bx = 0; bx < nbox; ++bx)
-                        tma_load_2d_pair(sb + bx * PAIR_BOX_ROWS * 128, &P.b, kb * 128, brow + bx * PAIR_BOX_ROWS, fb,
-                                         pol_x);
                     if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
@@ -223,12 +248,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
                 mbar_wait_bounded(drain, 0, &dummy, 100000000ull);
             }
         }
-    } else {
+    } else if (warp >= PAIR8_EPI_BEGIN) {
         // ---------------------------------------------------- epilogue: promotion + final (both CTAs)
-        const int q = warp & 3;                 // TMEM lane quarter: rows q*32 .. q*32+31
-        const int grp = (warp - 2) >> 2;        // column group: chunks c0 = 32*grp + 64*c
-        const int wi = warp - 2;
-        float* my_sc = sc_rows + wi * 64;
+        constexpr int NCH = PAIR8_NCH, NGRP = PAIR8_NGRP;
+        const int wi = warp - PAIR8_EPI_BEGIN;
+        const int q = wi & 3;                   // TMEM lane quarter (warp % 4): rows q*32 .. q*32+31
+        const int grp = wi >> 2;                // column group: chunks c0 = 32*grp + 32*NGRP*c
+        float* my_sc = sc_rows + wi * GCOLS;
         const uint32_t pempty0 = mapa_shared(smem_u32(&pempty[0]), 0);
         const uint32_t xmax_peer = mapa_shared(smem_u32(xmax), rank ^ 1u);
         const uint32_t xbar_peer = mapa_shared(smem_u32(&xbar[0]), rank ^ 1u);
@@ -252,49 +278,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
                 rb = 2 * it.m + (int)rank;
             }
             const size_t sbase = it.shared ? 0 : (size_t)it.g * a_rb;
-            float acc[2][32];
+            const bool any = 32 * grp < it.nvalid;  // warp-uniform: this warp has columns
+            float acc[NCH][32];
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
+            for (int c = 0; c < NCH; ++c)
 #pragma unroll
                 for (int j = 0; j < 32; ++j) acc[c][j] = 0.0f;
-            auto load_scales = [&](int kb, float& w, float (&xs)[2]) {
+            auto load_scales = [&](int kb, float& w, float (&xs)[NCH]) {
                 w = rb < a_rb ? __ldg(&sa[(sbase + rb) * KB + kb]) : 0.0f;
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const int col = 32 * grp + 64 * c + lane;
+                for (int c = 0; c < NCH; ++c) {
+                    const int col = 32 * grp + 32 * NGRP * c + lane;
                     xs[c] = col < it.nvalid ? __ldg(&P.sbT[(size_t)kb * P.sb_ld + it.row0 + col]) : 0.0f;
                 }
             };
-            float nw, nxs[2];
+            float nw, nxs[NCH];
             load_scales(0, nw, nxs);
             for (int kb = 0; kb < KB; ++kb) {
+                // this block's scales were loaded one block ahead; the next block's go out now
                 const float sw = nw;
-                const float xs0 = nxs[0], xs1 = nxs[1];
+                float xs[NCH];
+#pragma unroll
+                for (int c = 0; c < NCH; ++c) xs[c] = nxs[c];
                 if (kb + 1 < KB) load_scales(kb + 1, nw, nxs);
                 if (!mbar_wait_bounded(&pfull[pb], pb_phase, abort_flag)) { alive = false; break; }
                 tc_fence_after();
                 const uint32_t t0 = tmem_base + (uint32_t)(pb * C::P_COLS) + ((uint32_t)(q * 32) << 16);
-                const int c0a = 32 * grp, c0b = 32 * grp + 64;
-                if (c0a < it.nvalid) {
-                    my_sc[lane] = sw * xs0;
-                    my_sc[32 + lane] = sw * xs1;
+                if (any) {
+#pragma unroll
+                    for (int c = 0; c < NCH; ++c) my_sc[c * 32 + lane] = sw * xs[c];
                     __syncwarp();
-                    float p0[32], p1[32];
-                    tmem_ld32x2(t0 + (uint32_t)c0a, t0 + (uint32_t)c0b, p0, p1);
-                    const bool two = c0b < it.nvalid;
+                    // every chunk of the warp's columns in one go (columns past the item's
+                    // rows hold stale sums of this buffer and are not used)
+                    float p[NCH][32];
+                    if constexpr (NCH == 2) tmem_ld32x2(t0 + (uint32_t)(32 * grp), t0 + (uint32_t)(32 * grp + 32 * NGRP), p[0], p[1]);
+                    else tmem_ld32(t0 + (uint32_t)(32 * grp), p[0]);
 #pragma unroll
                     for (int j = 0; j < 32; j += 4) {
-                        const float4 s0 = *reinterpret_cast<const float4*>(my_sc + j);
-                        fma2(acc[0][j + 0], acc[0][j + 1], p0[j + 0], p0[j + 1], s0.x, s0.y);
-                        fma2(acc[0][j + 2], acc[0][j + 3], p0[j + 2], p0[j + 3], s0.z, s0.w);
-                        if (two) {
-                            const float4 s1 = *reinterpret_cast<const float4*>(my_sc + 32 + j);
-                            fma2(acc[1][j + 0], acc[1][j + 1], p1[j + 0], p1[j + 1], s1.x, s1.y);
-                            fma2(acc[1][j + 2], acc[1][j + 3], p1[j + 2], p1[j + 3], s1.z, s1.w);
+#pragma unroll
+                        for (int c = 0; c < NCH; ++c) {
+                            if (c == 0 || 32 * grp + 32 * NGRP * c < it.nvalid) {
+                                const float4 sv = *reinterpret_cast<const float4*>(my_sc + c * 32 + j);
+                                fma2(acc[c][j + 0], acc[c][j + 1], p[c][j + 0], p[c][j + 1], sv.x, sv.y);
+                                fma2(acc[c][j + 2], acc[c][j + 3], p[c][j + 2], p[c][j + 3], sv.z, sv.w);
+                            }
                         }
                     }
-                    __syncwarp();
+                    __syncwarp();  // my_sc is rewritten for the next block
                 }
+                // the partial is promoted: hand the buffer back to the MMA issuer (handing it
+                // back right after the TMEM load, before the FMAs, measured the same)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(pempty0 + (uint32_t)(pb * 8));
@@ -313,17 +346,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
                 if (q >= 2) {
                     const int fl = (q - 2) * 32 + lane;
 #pragma unroll
-                    for (int c = 0; c < 2; ++c)
+                    for (int c = 0; c < NCH; ++c)
 #pragma unroll
                         for (int j = 0; j < 32; ++j) xg[fl * C::XUP_STRIDE + c * 32 + j] = acc[c][j];
                 }
                 named_bar_sync(2 + grp, 128);
                 // (2) h = SiLU(gate) * up; per-warp column maxima over its 32 features
-                float* cm = cmax + grp * 128;  // [2 chunks][2 gate warps][32 columns]
+                float* cm = cmax + grp * (NCH * 2 * 32);  // [chunks][2 gate warps][32 columns]
                 if (q < 2) {
                     const int fl = q * 32 + lane;
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
+                    for (int c = 0; c < NCH; ++c) {
 #pragma unroll
                         for (int j = 0; j < 32; ++j) acc[c][j] = silu_mul(acc[c][j], xg[fl * C::XUP_STRIDE + c * 32 + j]);
                         float m[32];
@@ -346,36 +379,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
                 // (3) the block's 128 features span both CTAs: exchange the 64-feature
                 //     maxima with the peer, then scale = amax / 448 per token row
                 if (q == 0) {
-                    float lm[2];
+                    float lm[NCH];
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
+                    for (int c = 0; c < NCH; ++c) {
                         lm[c] = fmaxf(cm[(c * 2) * 32 + lane], cm[(c * 2 + 1) * 32 + lane]);
-                        st_cluster_f32(xmax_peer + (uint32_t)((par * 128 + grp * 64 + c * 32 + lane) * 4), lm[c]);
+                        st_cluster_f32(xmax_peer + (uint32_t)(((par * NGRP + grp) * GCOLS + c * 32 + lane) * 4), lm[c]);
                     }
                     __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster_release(xbar_peer + (uint32_t)((par * 2 + grp) * 8));
-                    const bool got = mbar_wait_cluster_bounded(&xbar[par * 2 + grp], x_phase[par], abort_flag);
-                    float* si = sinv + grp * 64;
+                    if (lane == 0) mbar_arrive_cluster_release(xbar_peer + (uint32_t)((par * NGRP + grp) * 8));
+                    const bool got = mbar_wait_cluster_bounded(&xbar[par * NGRP + grp], x_phase[par], abort_flag);
+                    float* si = sinv + grp * GCOLS;
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        const float amax = got ? fmaxf(lm[c], xmax[par * 128 + grp * 64 + c * 32 + lane]) : 0.0f;
+                    for (int c = 0; c < NCH; ++c) {
+                        const float amax = got ? fmaxf(lm[c], xmax[(par * NGRP + grp) * GCOLS + c * 32 + lane]) : 0.0f;
                         const float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
                         si[c * 32 + lane] = 1.0f / scale;
-                        const int col = 32 * grp + 64 * c + lane;
+                        const int col = 32 * grp + 32 * NGRP * c + lane;
                         if (leader && col < it.nvalid) P.hsT[(size_t)it.m * P.hs_ld + it.row0 + col] = scale;
                     }
                     if (lane == 0) warp_ok[wi] = got ? 1 : 0;
                 }
                 x_phase[par] ^= 1u;
                 named_bar_sync(2 + grp, 128);
-                if (!warp_ok[4 * grp + 2]) { alive = false; break; }  // the q0 warp is warp 4 + 4 * grp
+                if (!warp_ok[4 * grp]) { alive = false; break; }  // the group's q0 warp
                 // (4) e4m3 codes of h, one byte per (token row, feature)
                 if (q < 2) {
                     const int f = it.m * 128 + (int)rank * 64 + q * 32 + lane;
-                    const float* si = sinv + grp * 64;
+                    const float* si = sinv + grp * GCOLS;
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        const int c0 = 32 * grp + 64 * c;
+                    for (int c = 0; c < NCH; ++c) {
+                        const int c0 = 32 * grp + 32 * NGRP * c;
                         if (c0 < it.nvalid) {
                             uint8_t* dst = P.hq + (size_t)(it.row0 + c0) * P.ldh + f;
 #pragma unroll
@@ -395,8 +428,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
                 const int f = it.m * 256 + (int)rank * 128 + q * 32 + lane;
                 const bool okf = f < P.ldy;
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const int c0 = 32 * grp + 64 * c;
+                for (int c = 0; c < NCH; ++c) {
+                    const int c0 = 32 * grp + 32 * NGRP * c;
                     if (c0 < it.nvalid) {
                         // this lane's permuted row, handed to the other lanes by shuffles
                         const bool okr = c0 + lane < it.nvalid;

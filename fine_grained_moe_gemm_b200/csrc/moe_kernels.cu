@@ -956,7 +956,7 @@ static cudaError_t launch_gemm2_fp8_t(const GemmArgs* args, int grid, cudaStream
         attr_set[dev].store(true, std::memory_order_relaxed);
     }
     note_launch();
-    moe_gemm2_fp8_kernel<MODE><<<grid, GEMM_THREADS, Gemm2Fp8Cfg::SMEM_BYTES, s>>>(*args);
+    moe_gemm2_fp8_kernel<MODE><<<grid, PAIR8_THREADS, Gemm2Fp8Cfg::SMEM_BYTES, s>>>(*args);
     return cudaGetLastError();
 }
 
