@@ -115,6 +115,12 @@ def _configure(L):
     L.moe_status_string.restype = ctypes.c_char_p
     L.moe_status_string.argtypes = [I]
     L.moe_abi_version.restype = I
+    L.moe_ep_packed_row_bytes.restype = ctypes.c_size_t
+    L.moe_ep_packed_row_bytes.argtypes = [ctypes.POINTER(MoeConfig)]
+    L.moe_ep_dispatch_packed.restype = I
+    L.moe_ep_dispatch_packed.argtypes = [ctypes.POINTER(MoeConfig), I, I, P, P, P, I, P, P, P, P]
+    L.moe_ep_unpack.restype = I
+    L.moe_ep_unpack.argtypes = [ctypes.POINTER(MoeConfig), I, P, P, P, P, P]
     L.moe_forward_noalloc.restype = I
     L.moe_forward_noalloc.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, I, P, I, I, P]
     L.moe_debug_build.restype = I
@@ -398,6 +404,45 @@ def moe_ep_dispatch(cfg: MoeConfig, n_ranks: int, topk_idx, topk_w, x, send_coun
     _check(lib().moe_ep_dispatch(ctypes.byref(cfg), int(n_ranks), _p(topk_idx), _p(topk_w), _p(x), T,
                                  _p(send_counts), _p(send_offsets), _p(send_tok), _p(send_x), _p(send_idx),
                                  _p(send_w), _stream(stream)), "moe_ep_dispatch")
+
+
+def ep_packed_row_bytes(cfg: MoeConfig) -> int:
+    """Bytes of one packed dispatch row: bf16 x | int32 ids | fp32 weights, padded to 16."""
+    return int(lib().moe_ep_packed_row_bytes(ctypes.byref(cfg)))
+
+
+def moe_ep_dispatch_packed(cfg: MoeConfig, n_ranks: int, capacity: int, topk_idx, topk_w, x, send_counts, send_tok,
+                           packed, stream=None):
+    """Fixed-capacity packed dispatch: rank q's rows at slots [q*capacity, q*capacity + send_counts[q]) of
+    ``packed`` [n_ranks*capacity, ep_packed_row_bytes] uint8 and ``send_tok`` [n_ranks*capacity] int32; padding
+    slots have token -1 and expert ids -1."""
+    T = x.shape[0]
+    for n, t in (("topk_idx", topk_idx), ("topk_w", topk_w), ("x", x), ("send_counts", send_counts),
+                 ("send_tok", send_tok), ("packed", packed)):
+        _dev(t, n)
+    k, slots = cfg.top_k, n_ranks * capacity
+    _shape(topk_idx, "topk_idx", (T, k), (torch.int32,))
+    _shape(topk_w, "topk_w", (T, k), (torch.float32,))
+    _shape(x, "x", (T, cfg.d), _ACT.get(cfg.act_dtype, ()))
+    _shape(send_counts, "send_counts", (n_ranks,), (torch.int32,))
+    _shape(send_tok, "send_tok", (slots,), (torch.int32,))
+    _shape(packed, "packed", (slots, ep_packed_row_bytes(cfg)), (torch.uint8,))
+    _check(lib().moe_ep_dispatch_packed(ctypes.byref(cfg), int(n_ranks), int(capacity), _p(topk_idx), _p(topk_w),
+                                        _p(x), T, _p(send_counts), _p(send_tok), _p(packed), _stream(stream)),
+           "moe_ep_dispatch_packed")
+
+
+def moe_ep_unpack(cfg: MoeConfig, packed, x_rows, topk_idx, topk_w, stream=None):
+    """Packed rows -> x_rows [n, d] bf16, topk_idx / topk_w [n, k] (padding rows: ids -1)."""
+    for n, t in (("packed", packed), ("x_rows", x_rows), ("topk_idx", topk_idx), ("topk_w", topk_w)):
+        _dev(t, n)
+    n = packed.shape[0]
+    _shape(packed, "packed", (n, ep_packed_row_bytes(cfg)), (torch.uint8,))
+    _shape(x_rows, "x_rows", (n, cfg.d), (torch.bfloat16,))
+    _shape(topk_idx, "topk_idx", (n, cfg.top_k), (torch.int32,))
+    _shape(topk_w, "topk_w", (n, cfg.top_k), (torch.float32,))
+    _check(lib().moe_ep_unpack(ctypes.byref(cfg), n, _p(packed), _p(x_rows), _p(topk_idx), _p(topk_w),
+                               _stream(stream)), "moe_ep_unpack")
 
 
 def experts_routed_workspace_size(cfg: MoeConfig, n_local: int, n_rows: int) -> int:

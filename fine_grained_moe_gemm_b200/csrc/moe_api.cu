@@ -708,6 +708,45 @@ moe_status moe_ep_dispatch(const moe_config* cfg, int n_ranks, const int32_t* to
                                           (cudaStream_t)stream));
 }
 
+size_t moe_ep_packed_row_bytes(const moe_config* cfg) {
+    if (check_config(cfg) != MOE_OK) return 0;
+    return align_up((size_t)cfg->d * 2 + (size_t)cfg->top_k * 8, 16);
+}
+
+moe_status moe_ep_dispatch_packed(const moe_config* cfg, int n_ranks, int capacity, const int32_t* topk_idx,
+                                  const float* topk_w, const void* x, int T, int32_t* send_counts, int32_t* send_tok,
+                                  void* packed, moe_stream_t stream) {
+    NvtxRange nvtx_call("moe_ep_dispatch_packed");
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (T < 0 || capacity < T || capacity < 1 || n_ranks < 1 || n_ranks > 32 || cfg->n_experts % n_ranks != 0 ||
+        (long long)n_ranks * capacity > INT32_MAX)
+        return MOE_ERR_INVALID_ARG;
+    if (!send_counts || !send_tok || !packed || !aligned16(packed)) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!topk_idx || !topk_w || !x || !aligned16(x))) return MOE_ERR_INVALID_ARG;
+    DevInfo di;
+    if ((st = check_device(&di)) != MOE_OK) return st;
+    return cuda_status(launch_ep_dispatch_packed(topk_idx, topk_w, T, cfg->top_k, cfg->n_experts, n_ranks, capacity,
+                                                 x, cfg->act_dtype == MOE_F32, cfg->d, send_counts, send_tok,
+                                                 static_cast<uint8_t*>(packed), (int)moe_ep_packed_row_bytes(cfg),
+                                                 (cudaStream_t)stream));
+}
+
+moe_status moe_ep_unpack(const moe_config* cfg, int n_rows, const void* packed, void* x_rows, int32_t* topk_idx,
+                         float* topk_w, moe_stream_t stream) {
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (n_rows < 0) return MOE_ERR_INVALID_ARG;
+    if (n_rows == 0) return MOE_OK;
+    if (!packed || !x_rows || !topk_idx || !topk_w || !aligned16(packed) || !aligned16(x_rows))
+        return MOE_ERR_INVALID_ARG;
+    DevInfo di;
+    if ((st = check_device(&di)) != MOE_OK) return st;
+    return cuda_status(launch_ep_unpack(static_cast<const uint8_t*>(packed), n_rows, (int)moe_ep_packed_row_bytes(cfg),
+                                        cfg->d, cfg->top_k, static_cast<__nv_bfloat16*>(x_rows), topk_idx, topk_w,
+                                        (cudaStream_t)stream));
+}
+
 size_t moe_experts_routed_workspace_size(const moe_config* cfg, int n_local, int n_rows_max) {
     moe_config c;
     if (!local_cfg(cfg, n_local, &c) || n_rows_max < 0) return 0;

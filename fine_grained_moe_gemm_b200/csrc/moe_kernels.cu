@@ -751,21 +751,29 @@ __global__ void __launch_bounds__(EP_THREADS) ep_count_kernel(const int32_t* __r
 }
 
 // one CTA per rank: its offset and its send rows' origin tokens, in token order
+// capacity > 0: rank r's rows start at r * capacity (fixed-capacity layout; offsets
+// is not written) and its unused slots get token -1
 __global__ void __launch_bounds__(EP_THREADS) ep_place_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
                                                               int epr, int R, const int32_t* __restrict__ counts,
                                                               int32_t* __restrict__ offsets,
-                                                              int32_t* __restrict__ send_tok) {
+                                                              int32_t* __restrict__ send_tok, int capacity) {
     __shared__ int wsum[EP_THREADS / 32 + 1];
     __shared__ int base_s;
     const int r = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (threadIdx.x == 0) {
         int o = 0;
-        for (int q = 0; q < r; ++q) o += counts[q];
+        if (capacity > 0) {
+            o = r * capacity;
+        } else {
+            for (int q = 0; q < r; ++q) o += counts[q];
+            offsets[r] = o;
+            if (r == R - 1) offsets[R] = o + counts[r];
+        }
         base_s = o;
-        offsets[r] = o;
-        if (r == R - 1) offsets[R] = o + counts[r];
     }
     __syncthreads();
+    if (capacity > 0)
+        for (int j = counts[r] + threadIdx.x; j < capacity; j += EP_THREADS) send_tok[(size_t)r * capacity + j] = -1;
     int base = base_s;
     for (int t0 = 0; t0 < T; t0 += EP_THREADS) {
         const int t = t0 + threadIdx.x;
@@ -804,6 +812,64 @@ __global__ void __launch_bounds__(256) ep_rows_kernel(const int32_t* __restrict_
     }
 }
 
+// Packed dispatch rows (fixed-capacity layout): row r = bf16 x [d] | ids int32 [k] |
+// weights fp32 [k] | padding to row_bytes.  One CTA per row; a padding slot (token
+// -1) gets ids -1 (its x and weights are left as they are).
+__global__ void __launch_bounds__(128) ep_pack_kernel(const int32_t* __restrict__ idx, const float* __restrict__ w,
+                                                      int k, const void* __restrict__ x, int x_f32, int d,
+                                                      const int32_t* __restrict__ send_tok,
+                                                      uint8_t* __restrict__ packed, int row_bytes) {
+    const int r = blockIdx.x;
+    const int t = send_tok[r];
+    uint8_t* row = packed + (size_t)r * row_bytes;
+    int32_t* ids = reinterpret_cast<int32_t*>(row + (size_t)d * 2);
+    float* ws = reinterpret_cast<float*>(row + (size_t)d * 2 + (size_t)k * 4);
+    if (t < 0) {
+        for (int j = threadIdx.x; j < k; j += blockDim.x) ids[j] = -1;
+        return;
+    }
+    for (int j = threadIdx.x; j < k; j += blockDim.x) {
+        ids[j] = idx[(size_t)t * k + j];
+        ws[j] = w[(size_t)t * k + j];
+    }
+    uint4* dst = reinterpret_cast<uint4*>(row);
+    const int nvec = d / 8;  // 8 bf16 per 16 bytes
+    if (x_f32) {
+        const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(x) + (size_t)t * d);
+        for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+            const float4 a = src[2 * v], b = src[2 * v + 1];
+            __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y), p1 = __floats2bfloat162_rn(a.z, a.w);
+            __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y), p3 = __floats2bfloat162_rn(b.z, b.w);
+            dst[v] = make_uint4(*reinterpret_cast<uint32_t*>(&p0), *reinterpret_cast<uint32_t*>(&p1),
+                                *reinterpret_cast<uint32_t*>(&p2), *reinterpret_cast<uint32_t*>(&p3));
+        }
+    } else {
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + (size_t)t * d);
+        for (int v = threadIdx.x; v < nvec; v += blockDim.x) dst[v] = src[v];
+    }
+}
+
+// received packed rows -> the three arrays moe_experts_routed reads; one CTA per row
+// (a padding row's ids stay -1, so its slots are skipped there)
+__global__ void __launch_bounds__(128) ep_unpack_kernel(const uint8_t* __restrict__ packed, int row_bytes, int d,
+                                                        int k, __nv_bfloat16* __restrict__ x_rows,
+                                                        int32_t* __restrict__ ids_out, float* __restrict__ w_out) {
+    const int r = blockIdx.x;
+    const uint8_t* row = packed + (size_t)r * row_bytes;
+    const int32_t* ids = reinterpret_cast<const int32_t*>(row + (size_t)d * 2);
+    const float* ws = reinterpret_cast<const float*>(row + (size_t)d * 2 + (size_t)k * 4);
+    bool live = false;
+    for (int j = 0; j < k; ++j) live |= ids[j] >= 0;  // uniform over the block
+    for (int j = threadIdx.x; j < k; j += blockDim.x) {
+        ids_out[(size_t)r * k + j] = ids[j];
+        w_out[(size_t)r * k + j] = live ? ws[j] : 0.0f;
+    }
+    if (!live) return;  // nothing reads a padding row's x
+    const uint4* src = reinterpret_cast<const uint4*>(row);
+    uint4* dst = reinterpret_cast<uint4*>(x_rows + (size_t)r * d);
+    for (int v = threadIdx.x; v < d / 8; v += blockDim.x) dst[v] = src[v];
+}
+
 // combine: acc[send_tok[r], :] += back[r, :] (the partial sums the ranks returned)
 __global__ void __launch_bounds__(256) ep_combine_kernel(const float* __restrict__ back,
                                                          const int32_t* __restrict__ send_tok, int n_rows, int T,
@@ -814,6 +880,7 @@ __global__ void __launch_bounds__(256) ep_combine_kernel(const float* __restrict
         const size_t r = i / d4;
         const int c = (int)(i - r * d4) * 4;
         const int t = send_tok[r];
+        if (t == -1) continue;             // a padding slot of the fixed-capacity layout
         if ((unsigned)t >= (unsigned)T) {  // not a token of this batch: flagged and skipped
             set_dev_error(MOE_DEVERR_BAD_ROWS);
             continue;
@@ -1136,7 +1203,7 @@ cudaError_t launch_ep_dispatch(const int32_t* idx, const float* w, int T, int k,
     note_launch();
     ep_count_kernel<<<R, EP_THREADS, 0, s>>>(idx, T, k, E, epr, counts);
     note_launch();
-    ep_place_kernel<<<R, EP_THREADS, 0, s>>>(idx, T, k, E, epr, R, counts, offsets, send_tok);
+    ep_place_kernel<<<R, EP_THREADS, 0, s>>>(idx, T, k, E, epr, R, counts, offsets, send_tok, 0);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || T == 0) return e;
     const int max_rows = T * (k < R ? k : R);
@@ -1145,6 +1212,26 @@ cudaError_t launch_ep_dispatch(const int32_t* idx, const float* w, int T, int k,
     grid = grid < n_sm * 4 ? grid : n_sm * 4;
     note_launch();
     ep_rows_kernel<<<grid, 256, 0, s>>>(idx, w, k, send_tok, offsets + R, send_idx, send_w);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ep_dispatch_packed(const int32_t* idx, const float* w, int T, int k, int E, int R, int capacity,
+                                      const void* x, bool x_f32, int d, int32_t* counts, int32_t* send_tok,
+                                      uint8_t* packed, int row_bytes, cudaStream_t s) {
+    const int epr = E / R;
+    note_launch();
+    ep_count_kernel<<<R, EP_THREADS, 0, s>>>(idx, T, k, E, epr, counts);
+    note_launch();
+    ep_place_kernel<<<R, EP_THREADS, 0, s>>>(idx, T, k, E, epr, R, counts, nullptr, send_tok, capacity);
+    note_launch();
+    ep_pack_kernel<<<R * capacity, 128, 0, s>>>(idx, w, k, x, x_f32 ? 1 : 0, d, send_tok, packed, row_bytes);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ep_unpack(const uint8_t* packed, int n_rows, int row_bytes, int d, int k, __nv_bfloat16* x_rows,
+                             int32_t* ids, float* w, cudaStream_t s) {
+    note_launch();
+    ep_unpack_kernel<<<n_rows, 128, 0, s>>>(packed, row_bytes, d, k, x_rows, ids, w);
     return cudaGetLastError();
 }
 

@@ -17,14 +17,28 @@ One forward on every rank, in the same order on all of them:
 Every step but the exchange runs in the library's kernels; the exchange is
 torch.distributed's all-to-all (NCCL between GPUs, gloo on CPU).  The result
 equals moe_forward's on the same tokens up to the order of fp32 additions.
+
+Two forms of the same layer:
+  moe_forward_ep  variable-size exchange: the row counts go to the host, so only
+                  the rows that exist cross the link (large batches); it syncs
+                  the host once per forward and allocates per call.
+  EpLayer         fixed-capacity exchange, for decode-sized batches: every
+                  buffer is allocated once for up to T_max tokens per rank; rank
+                  q's rows travel in a block of T_max packed rows (x, expert ids
+                  and weights in one row; unused slots marked by ids -1), so both
+                  all-to-alls have equal splits known in advance, nothing waits
+                  on the host, and a forward can be captured in a CUDA graph.
+                  The price is padding: each block is T_max rows whatever the
+                  count.
 """
 from __future__ import annotations
 
 import torch
 import torch.distributed as dist
 
-from . import (MOE_BF16, MOE_E4M3, MoeConfig, dense_workspace_size, ep_max_send_rows, experts_routed_workspace_size,
-               moe_dense_ffn, moe_ep_combine, moe_ep_dispatch, moe_experts_routed, moe_route)
+from . import (MOE_BF16, MOE_E4M3, MoeConfig, dense_workspace_size, ep_max_send_rows, ep_packed_row_bytes,
+               experts_routed_workspace_size, moe_dense_ffn, moe_ep_combine, moe_ep_dispatch, moe_ep_dispatch_packed,
+               moe_ep_unpack, moe_experts_routed, moe_route)
 
 
 def exchange_counts(send_counts: torch.Tensor, group=None) -> torch.Tensor:
@@ -103,3 +117,69 @@ def moe_forward_ep(cfg: MoeConfig, w_router, local_weights: dict, shared_weights
                       shared_weights.get("s_gate"), shared_weights.get("s_up"), shared_weights.get("s_down"),
                       workspace=dws)
         moe_ep_combine(back, send_tok, y_acc, y, residual)
+
+
+class EpLayer:
+    """The expert-parallel layer with a device-resident, fixed-capacity exchange (see the module docstring).
+
+    Every rank of ``group`` builds one with the same ``T_max`` and calls :meth:`forward` together.  Buffers are
+    allocated here, once; a forward allocates nothing, never reads a count on the host, and its two all-to-alls
+    have equal splits (T_max packed rows per peer there, T_max fp32 rows back), so on NCCL it can be captured in a
+    CUDA graph.  ``shared_hidden`` / ``shared_e4m3`` size the shared expert's workspace."""
+
+    def __init__(self, cfg: MoeConfig, T_max: int, device, group=None, shared_hidden: int | None = None,
+                 shared_e4m3: bool = False):
+        if cfg.n_shared != 1:
+            raise ValueError("the expert-parallel layer takes one shared expert")
+        self.cfg, self.T_max, self.group = cfg, int(T_max), group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        self.lo, self.n_local = expert_block(cfg, self.rank, self.world)
+        d, k, E = cfg.d, cfg.top_k, cfg.n_experts
+        slots = self.world * self.T_max
+        rb = ep_packed_row_bytes(cfg)
+        dev = torch.device(device)
+        f32, i32 = torch.float32, torch.int32
+        self.logits = torch.empty((self.T_max, E), dtype=f32, device=dev)
+        self.idx = torch.empty((self.T_max, k), dtype=i32, device=dev)
+        self.w = torch.empty((self.T_max, k), dtype=f32, device=dev)
+        self.counts = torch.empty(self.world, dtype=i32, device=dev)
+        self.send_tok = torch.empty(slots, dtype=i32, device=dev)
+        self.send = torch.empty((slots, rb), dtype=torch.uint8, device=dev)
+        self.recv = torch.empty((slots, rb), dtype=torch.uint8, device=dev)
+        self.recv_x = torch.empty((slots, d), dtype=torch.bfloat16, device=dev)
+        self.recv_idx = torch.empty((slots, k), dtype=i32, device=dev)
+        self.recv_w = torch.empty((slots, k), dtype=f32, device=dev)
+        self.recv_y = torch.empty((slots, d), dtype=f32, device=dev)
+        self.back = torch.empty((slots, d), dtype=f32, device=dev)
+        self.y_acc = torch.empty((self.T_max, d), dtype=f32, device=dev)
+        self.ws = torch.empty(max(experts_routed_workspace_size(cfg, self.n_local, slots), 1), dtype=torch.uint8,
+                              device=dev)
+        hs = cfg.shared_hidden if shared_hidden is None else shared_hidden
+        wdt = MOE_E4M3 if shared_e4m3 else MOE_BF16
+        self.dws = torch.empty(max(dense_workspace_size(d, hs, cfg.act_dtype, wdt, self.T_max), 1),
+                               dtype=torch.uint8, device=dev)
+
+    def forward(self, w_router, local_weights: dict, shared_weights: dict, bias, x, y, residual=None):
+        """y = MoE(x) (+ residual) for this rank's tokens x [T, d], T <= T_max; arguments as moe_forward_ep."""
+        cfg, T = self.cfg, x.shape[0]
+        if T > self.T_max:
+            raise ValueError(f"{T} tokens, the layer was built for at most {self.T_max}")
+        # (1) routing of this rank's tokens, (2) dispatch into fixed-capacity packed rows
+        moe_route(cfg, x, w_router, self.logits[:T], bias, self.idx[:T], self.w[:T])
+        moe_ep_dispatch_packed(cfg, self.world, self.T_max, self.idx[:T], self.w[:T], x, self.counts, self.send_tok,
+                               self.send)
+        # (3) rows to their ranks: equal blocks of T_max rows, no counts needed
+        dist.all_to_all_single(self.recv, self.send, group=self.group)
+        # (4) this rank's experts on every received slot (padding slots carry no local expert)
+        moe_ep_unpack(cfg, self.recv, self.recv_x, self.recv_idx, self.recv_w)
+        moe_experts_routed(cfg, local_weights, self.lo, self.n_local, self.recv_x, self.recv_idx, self.recv_w,
+                           self.recv_y, workspace=self.ws)
+        # (5) partial sums back, block for block
+        dist.all_to_all_single(self.back, self.recv_y, group=self.group)
+        # (6) the shared expert on this rank's tokens, (7) combine (padding slots skipped)
+        if T:
+            moe_dense_ffn(shared_weights["w_gate"], shared_weights["w_up"], shared_weights["w_down"], x,
+                          self.y_acc[:T], shared_weights.get("s_gate"), shared_weights.get("s_up"),
+                          shared_weights.get("s_down"), workspace=self.dws)
+            moe_ep_combine(self.back, self.send_tok, self.y_acc[:T], y, residual)

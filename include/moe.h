@@ -361,6 +361,32 @@ MOE_API moe_status moe_ep_dispatch(const moe_config* cfg, int n_ranks, const int
                                    int32_t* send_tok, void* send_x, int32_t* send_idx, float* send_w,
                                    moe_stream_t stream);
 
+/* Fixed-capacity, packed dispatch: the same rows as moe_ep_dispatch, laid out so
+ * that the exchange needs no row counts on the host (equal-sized all-to-all
+ * blocks, capturable in a CUDA graph).  Rank q's rows occupy slots
+ * [q * capacity, q * capacity + send_counts[q]) in ascending token order; the
+ * other slots of its block are padding.  Each slot is one packed row of
+ * moe_ep_packed_row_bytes(cfg) bytes:
+ *   bf16 x [d] (fp32 x rounded to bf16) | int32 expert ids [k] | fp32 weights [k] | padding to 16 B
+ * a padding slot has send_tok = -1 and all k ids -1 (its x and weights are
+ * unspecified), so a receiver skips it without knowing the counts.
+ *   send_counts [n_ranks]       rows for each rank (for the caller's bookkeeping)
+ *   send_tok [n_ranks*capacity] origin token of each slot, -1 for padding
+ *   packed [n_ranks*capacity, row_bytes], 16-byte aligned
+ * capacity >= T (a token goes to a rank at most once) and the same on every
+ * rank.  Errors as moe_ep_dispatch. */
+MOE_API size_t moe_ep_packed_row_bytes(const moe_config* cfg);
+MOE_API moe_status moe_ep_dispatch_packed(const moe_config* cfg, int n_ranks, int capacity, const int32_t* topk_idx,
+                                          const float* topk_w, const void* x, int T, int32_t* send_counts,
+                                          int32_t* send_tok, void* packed, moe_stream_t stream);
+
+/* Received packed rows (n_rows of them, as moe_ep_dispatch_packed lays them
+ * out) into the inputs of moe_experts_routed: x_rows [n_rows, d] bf16,
+ * topk_idx / topk_w [n_rows, k].  Padding rows keep ids -1 (weights 0), which
+ * moe_experts_routed skips as foreign slots; their x rows are not written. */
+MOE_API moe_status moe_ep_unpack(const moe_config* cfg, int n_rows, const void* packed, void* x_rows,
+                                 int32_t* topk_idx, float* topk_w, moe_stream_t stream);
+
 /* Device workspace bytes of moe_experts_routed for up to n_rows_max rows and a
  * block of n_local experts (0 on invalid arguments). */
 MOE_API size_t moe_experts_routed_workspace_size(const moe_config* cfg, int n_local, int n_rows_max);
@@ -384,7 +410,8 @@ MOE_API moe_status moe_experts_routed(const moe_config* cfg, const moe_weights* 
  * atomics: a token's partial sums from the ranks it was sent to), then, with y
  * not NULL, y = bf16(y_acc + residual) ([T, d] bf16; residual bf16 [T, d] or
  * NULL, and may be y itself).  y_acc [T, d] fp32 holds the shared expert's output
- * on entry.  A send_tok entry outside [0, T) sets MOE_DEVERR_BAD_ROWS and its
+ * on entry.  A send_tok entry of -1 is a padding slot of the packed layout and
+ * is skipped; any other entry outside [0, T) sets MOE_DEVERR_BAD_ROWS and its
  * row is skipped.  d a multiple of 8; arrays 16-byte aligned. */
 MOE_API moe_status moe_ep_combine(int T, int d, int n_rows, const float* back_rows, const int32_t* send_tok,
                                   float* y_acc, void* y, const void* residual, moe_stream_t stream);

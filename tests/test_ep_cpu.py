@@ -224,3 +224,111 @@ def test_forward_ep_control_flow_gloo(tmp_path, world):
     port = _free_port()
     mp.spawn(_forward_rank, args=(world, port, str(tmp_path)), nprocs=world, join=True)
     assert all(open(tmp_path / f"f{r}").read() == "1" for r in range(world))
+
+
+# ----------------------------------------------------------------------------- fixed-capacity exchange
+
+def test_packed_entry_arguments(L):
+    cfg = cfg_of(WORKLOADS["decode"])
+    P = ctypes.c_void_p
+    assert L.moe_ep_packed_row_bytes(ctypes.byref(cfg)) == 2 * 7168 + 8 * 8          # 14400, a multiple of 16
+    tiny = cfg_of(WORKLOADS["tiny"])
+    assert L.moe_ep_packed_row_bytes(ctypes.byref(tiny)) == (2 * 256 + 8 * 4 + 15) // 16 * 16
+    dp = lambda R, cap, T, counts=P(16), packed=P(16): L.moe_ep_dispatch_packed(
+        ctypes.byref(cfg), R, cap, P(16), P(16), P(16), T, counts, P(16), packed, None)
+    assert dp(8, 3, 4) == moe.MOE_ERR_INVALID_ARG              # capacity below T
+    assert dp(0, 4, 4) == moe.MOE_ERR_INVALID_ARG              # no ranks
+    assert dp(3, 4, 4) == moe.MOE_ERR_INVALID_ARG              # 256 experts do not split over 3
+    assert dp(8, 4, 4, counts=None) == moe.MOE_ERR_INVALID_ARG
+    assert dp(8, 4, 4, packed=P(24)) == moe.MOE_ERR_INVALID_ARG  # misaligned rows
+    assert L.moe_ep_unpack(ctypes.byref(cfg), -1, P(16), P(16), P(16), P(16), None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_ep_unpack(ctypes.byref(cfg), 4, None, P(16), P(16), P(16), None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_ep_unpack(ctypes.byref(cfg), 0, None, None, None, None, None) == moe.MOE_OK
+
+
+def _packed_stand_ins(ep_mod):
+    """CPU stand-ins of the packed dispatch / unpack that follow the header's layout
+    (bf16 x | int32 ids | fp32 weights | padding; padding slots: token -1, ids -1)."""
+    def row_bytes(cfg):
+        return (2 * cfg.d + 8 * cfg.top_k + 15) // 16 * 16
+
+    def dispatch_packed(cfg, R, cap, idx, w, x, counts, send_tok, packed, stream=None):
+        d, k = cfg.d, cfg.top_k
+        c, tok = dispatch_def(idx.numpy(), cfg.n_experts, R)
+        counts.copy_(torch.from_numpy(c))
+        send_tok.fill_(-1)
+        packed.zero_()
+        ids_view = packed[:, 2 * d:2 * d + 4 * k]
+        ids_view.copy_(torch.full((packed.shape[0], k), -1, dtype=torch.int32).view(torch.uint8))
+        base = 0
+        for q in range(R):
+            for j in range(int(c[q])):
+                t = int(tok[base + j])
+                s = q * cap + j
+                send_tok[s] = t
+                packed[s, :2 * d] = x[t].to(torch.bfloat16).view(torch.uint8)
+                packed[s, 2 * d:2 * d + 4 * k] = idx[t].view(torch.uint8)
+                packed[s, 2 * d + 4 * k:2 * d + 8 * k] = w[t].view(torch.uint8)
+            base += int(c[q])
+
+    def unpack(cfg, packed, x_rows, idx, w, stream=None):
+        d, k = cfg.d, cfg.top_k
+        x_rows.copy_(packed[:, :2 * d].contiguous().view(torch.bfloat16))
+        idx.copy_(packed[:, 2 * d:2 * d + 4 * k].contiguous().view(torch.int32))
+        w.copy_(packed[:, 2 * d + 4 * k:2 * d + 8 * k].contiguous().view(torch.float32))
+        w[(idx < 0).all(1)] = 0.0
+
+    def combine(back, send_tok, y_acc, y=None, residual=None, stream=None):
+        keep = send_tok[: back.shape[0]] >= 0
+        y_acc.index_add_(0, send_tok[: back.shape[0]][keep].long(), back[keep])
+        if y is not None:
+            y.copy_((y_acc + (residual.float() if residual is not None else 0)).to(torch.bfloat16))
+
+    ep_mod.ep_packed_row_bytes = row_bytes
+    ep_mod.moe_ep_dispatch_packed, ep_mod.moe_ep_unpack, ep_mod.moe_ep_combine = dispatch_packed, unpack, combine
+
+
+def _ep_layer_rank(rank, world, port, out):
+    import datetime
+
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import fine_grained_moe_gemm_b200 as moe_pkg
+    from fine_grained_moe_gemm_b200 import ep
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    E, k, d = 16, 4, 32
+    cfg = moe_pkg.MoeConfig(d * 4, E, 4, 2, k, 128, 1, 128, 2.5)
+    cfg.d = d
+    _stand_ins(ep, E)
+    _packed_stand_ins(ep)
+    T_max = 9 + 5 * (world - 1)                               # the largest batch, the same on every rank
+    layer = ep.EpLayer(cfg, T_max, "cpu")
+    shared = {n: torch.empty((128, d), dtype=torch.bfloat16) for n in ("w_gate", "w_up", "w_down")}
+    ok = True
+    for step, T in enumerate((9 + 5 * rank, 3 + rank, T_max)):   # ranks differ in T; the blocks stay T_max rows
+        g = torch.Generator().manual_seed(7 + rank + 100 * step)
+        x = torch.randn((T, d), generator=g).to(torch.bfloat16)
+        y = torch.empty((T, d), dtype=torch.bfloat16)
+        layer.forward(None, {}, shared, torch.zeros(E), x, y)
+        xf = x.double()
+        top = torch.topk(xf.float()[:, :E], k, dim=1)
+        p = torch.sigmoid(top.values)
+        wts = (p / p.sum(1, keepdim=True)).double()
+        coef = (wts * (top.indices.double() + 1)).sum(1, keepdim=True)
+        ref = 0.5 * xf + 2.5 * coef * xf
+        ok &= bool(((y.double() - ref).abs() <= 2.0 ** -7 * ref.abs() + 1e-6).all())
+    dist.barrier()
+    dist.destroy_process_group()
+    with open(os.path.join(out, f"p{rank}"), "w") as f:
+        f.write(str(int(ok)))
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_ep_layer_control_flow_gloo(tmp_path, world):
+    """EpLayer.forward end to end on gloo ranks (equal-split all-to-alls of packed rows and of the fp32
+    results), three batches of different sizes through the same buffers, every token against its closed form."""
+    port = _free_port()
+    mp.spawn(_ep_layer_rank, args=(world, port, str(tmp_path)), nprocs=world, join=True)
+    assert all(open(tmp_path / f"p{r}").read() == "1" for r in range(world))
