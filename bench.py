@@ -46,7 +46,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel per launch, from one ncu capture, keyed by workload: (bytes, kernel
 # source hash the capture was taken at, how the figure was obtained).  A figure
 # is reported only while the kernel sources still hash to the recorded value.
-NCU_TRAFFIC: dict = {}
+NCU_TRAFFIC: dict = {
+    "profile_decode": (1_826_354_944, "e1cd8ed46c47add6",
+                       "ncu capture of this workload's gate/up GEMM: dram__bytes_read.sum + dram__bytes_write.sum"),
+    "decode": (8_587_015_424, "e1cd8ed46c47add6",
+               "ncu capture of the 31-weight-set decode-shaped case (profile_decode), reads scaled by the weight "
+               "sets streamed, 146 / 31, writes as captured"),
+}
 
 HBM_NOMINAL_GBS = 7700.0  # B200 (HGX) HBM3e nominal bandwidth, for context beside the measured copy peak
 
