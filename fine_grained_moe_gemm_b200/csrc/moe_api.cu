@@ -859,8 +859,9 @@ moe_status run_experts(const moe_config* cfg, const moe_weights* wt, const Works
             launch_gather_fp8(W.x_q, W.sx, d, T, W.row_tok, W.row_off + NG, rows_max, W.xq_perm, W.sxT, di.sm_count,
                               s) != cudaSuccess)
             return MOE_ERR_CUDA;
-    } else if (!direct_b && launch_gather(x, cfg->act_dtype == MOE_F32, d, T, W.row_tok, W.row_off + NG, rows_max,
-                                          W.x_perm, di.sm_count, s) != cudaSuccess) {
+    } else if (!direct_b && launch_scatter_rows(x, cfg->act_dtype == MOE_F32, d, T, k, W.inv,
+                                                cfg->n_shared ? W.row_off + E : nullptr, rows_max, W.x_perm,
+                                                di.sm_count, s) != cudaSuccess) {
         return MOE_ERR_CUDA;
     }
     mark(2);

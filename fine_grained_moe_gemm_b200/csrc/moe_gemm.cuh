@@ -120,9 +120,12 @@ __device__ __forceinline__ Item decode_item(const GemmArgs& P, int i) {
     it.shared = lo >= P.n_routed;
     it.K = it.shared ? P.K_shared : P.K_routed;
     if (kDebugChecks && P.rows_cap > 0) {
-        // checking build: the item's rows inside the permuted buffers and its weight
-        // tile inside the expert (every role decodes the same replacement)
+        // checking build: the group's rows agree with its item count, the item's rows
+        // lie inside the permuted buffers and its weight tile inside the expert
+        // (every role decodes the same replacement)
         const int mt = it.shared ? P.mt_shared : P.mt_routed;
+        const int n_items = __ldg(&P.item_off[lo + 1]) - __ldg(&P.item_off[lo]);
+        dbg_ok(n_items == nch * mt * it.n_splits);
         if (!dbg_ok(it.row0 >= 0 && it.nvalid >= 1 && it.row0 + it.nvalid <= P.rows_cap && it.m >= 0 && it.m < mt)) {
             it.row0 = 0;
             it.nvalid = min(BN, P.rows_cap);

@@ -496,6 +496,59 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const void* __restrict
     }
 }
 
+// Token-major form of the same copy: a CTA reads token t's row once (converting
+// fp32 to bf16 once) and writes it to the permuted rows of its (token, slot)
+// pairs, inv[t*k + j] (-1: the pair has no row here), and to its shared-expert
+// row shared_base + t.  Every x row is read once instead of once per row that
+// holds it, which matters when x does not stay in L2 between its copies.
+__global__ void __launch_bounds__(256) scatter_rows_kernel(const void* __restrict__ x, int x_f32, int d, int T, int k,
+                                                           const int32_t* __restrict__ inv,
+                                                           const int32_t* __restrict__ shared_base_dev, int rows_cap,
+                                                           __nv_bfloat16* __restrict__ xp) {
+    __shared__ int s_rows[33];  // top_k <= 32, + the shared-expert row
+    const int nvec = d / 8;     // 8 bf16 per 16-byte vector
+    const int shared_base = shared_base_dev ? *shared_base_dev : -1;
+    for (int t = blockIdx.x; t < T; t += gridDim.x) {
+        __syncthreads();  // the previous token's rows are no longer read
+        if (threadIdx.x <= k) {
+            int row = threadIdx.x < k ? inv[(size_t)t * k + threadIdx.x] : (shared_base >= 0 ? shared_base + t : -1);
+            // checking build: a row inside the permuted buffer (else it is skipped)
+            if (kDebugChecks && row >= 0 && !dbg_ok(row < rows_cap)) row = -1;
+            s_rows[threadIdx.x] = row;
+        }
+        __syncthreads();
+        for (int v0 = 0; v0 < nvec; v0 += 4 * 256) {
+            uint4 buf[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int v = v0 + j * 256 + threadIdx.x;
+                if (v >= nvec) break;
+                if (x_f32) {
+                    const float4* srcf = reinterpret_cast<const float4*>(static_cast<const float*>(x) + (size_t)t * d);
+                    const float4 a = srcf[2 * v], b = srcf[2 * v + 1];
+                    __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y), p1 = __floats2bfloat162_rn(a.z, a.w);
+                    __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y), p3 = __floats2bfloat162_rn(b.z, b.w);
+                    buf[j] = make_uint4(*reinterpret_cast<uint32_t*>(&p0), *reinterpret_cast<uint32_t*>(&p1),
+                                        *reinterpret_cast<uint32_t*>(&p2), *reinterpret_cast<uint32_t*>(&p3));
+                } else {
+                    buf[j] = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + (size_t)t * d)[v];
+                }
+            }
+            for (int jr = 0; jr <= k; ++jr) {
+                const int row = s_rows[jr];
+                if (row < 0) continue;  // uniform over the block
+                uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)row * d);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int v = v0 + j * 256 + threadIdx.x;
+                    if (v >= nvec) break;
+                    dst[v] = buf[j];
+                }
+            }
+        }
+    }
+}
+
 // ============================================================================ FP8 activations
 // "Teardown: DeepSeek-V3", section 10: activations scaled in 1x128 tiles.
 // One warp per (token, 128-channel block), 4 channels per lane:
@@ -1132,6 +1185,16 @@ cudaError_t launch_gather(const void* x, bool x_f32, int d, int n_tok, const int
     if (grid < 1) grid = 1;
     note_launch();
     gather_rows_kernel<<<grid, 256, 0, s>>>(x, x_f32 ? 1 : 0, d, n_tok, row_tok, n_rows_dev, max_rows, x_perm);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_rows(const void* x, bool x_f32, int d, int T, int k, const int32_t* inv,
+                                const int32_t* shared_base_dev, int rows_cap, __nv_bfloat16* x_perm, int n_sm,
+                                cudaStream_t s) {
+    int grid = T < n_sm * 8 ? T : n_sm * 8;
+    if (grid < 1) grid = 1;
+    note_launch();
+    scatter_rows_kernel<<<grid, 256, 0, s>>>(x, x_f32 ? 1 : 0, d, T, k, inv, shared_base_dev, rows_cap, x_perm);
     return cudaGetLastError();
 }
 

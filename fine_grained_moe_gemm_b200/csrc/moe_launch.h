@@ -113,6 +113,11 @@ cudaError_t launch_ep_combine(const float* back, const int32_t* send_tok, int n_
 // (checking build: row_tok entries against n_tok, the row count against max_rows)
 cudaError_t launch_gather(const void* x, bool x_f32, int d, int n_tok, const int32_t* row_tok,
                           const int32_t* n_rows_dev, int max_rows, __nv_bfloat16* x_perm, int n_sm, cudaStream_t s);
+// token-major copy into x_perm: token t's row to rows inv[t*k + j] (>= 0) and, when
+// shared_base_dev is set, to row *shared_base_dev + t
+cudaError_t launch_scatter_rows(const void* x, bool x_f32, int d, int T, int k, const int32_t* inv,
+                                const int32_t* shared_base_dev, int rows_cap, __nv_bfloat16* x_perm, int n_sm,
+                                cudaStream_t s);
 // q[t, :], sx[t, b]: per-token, per-128-channel e4m3 quantisation of bf16 x
 cudaError_t launch_quant_act(const __nv_bfloat16* x, int T, int d, uint8_t* q, float* sx, cudaStream_t s);
 // xpq[r, :] = xq[row_tok[r], :]; sxT[b][r] = sx[row_tok[r], b] for r < row_off[n_groups]
