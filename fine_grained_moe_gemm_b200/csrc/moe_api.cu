@@ -474,8 +474,9 @@ moe_status moe_forward_plan(const moe_config* cfg, int T, moe_dtype y_dtype, moe
     out->fp8 = p.fp8 ? 1 : 0;
     out->router_splits = p.router_parts;
     out->permute_ctas = p.permute_multi ? permute_blocks(T) : 1;
-    // router + selection, permutation, gather (+ quantisation), two GEMMs, bf16 cast
-    out->launches = 2 + (p.permute_multi ? 3 : 1) + (p.fp8 ? 2 : 1) + 2 + (y_dtype == MOE_BF16 ? 1 : 0);
+    // router + selection, permutation, copy into expert order (with the quantisation), two
+    // GEMMs, bf16 cast
+    out->launches = 2 + (p.permute_multi ? 3 : 1) + 1 + 2 + (y_dtype == MOE_BF16 ? 1 : 0);
     return MOE_OK;
 }
 
@@ -855,9 +856,10 @@ moe_status run_experts(const moe_config* cfg, const moe_weights* wt, const Works
     NvtxStages nv;
     nv.next(fp8 ? "moe.quantize+gather" : "moe.gather");
     if (fp8) {
-        if ((!act_quantised && launch_quant_act(static_cast<const __nv_bfloat16*>(x), T, d, W.x_q, W.sx, s) != cudaSuccess) ||
-            launch_gather_fp8(W.x_q, W.sx, d, T, W.row_tok, W.row_off + NG, rows_max, W.xq_perm, W.sxT, di.sm_count,
-                              s) != cudaSuccess)
+        if (launch_quant_scatter_fp8(act_quantised ? nullptr : static_cast<const __nv_bfloat16*>(x),
+                                     act_quantised ? W.x_q : nullptr, W.sx, d, T, k, W.inv,
+                                     cfg->n_shared ? W.row_off + E : nullptr, rows_max, W.xq_perm, W.sxT, di.sm_count,
+                                     s) != cudaSuccess)
             return MOE_ERR_CUDA;
     } else if (!direct_b && launch_scatter_rows(x, cfg->act_dtype == MOE_F32, d, T, k, W.inv,
                                                 cfg->n_shared ? W.row_off + E : nullptr, rows_max, W.x_perm,

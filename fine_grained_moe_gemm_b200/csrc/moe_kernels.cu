@@ -5,9 +5,10 @@
 //   permute_kernel        histogram / prefix sum / stable scatter by expert, and
 //                         the tile schedules of the grouped GEMMs (one CTA);
 //   permute_count/scan/scatter_kernel   the same over many CTAs (large T)
-//   gather_rows_kernel    x_perm = x[row_tok] (bf16)
+//   scatter_rows_kernel   x_perm written token-major (bf16)
+//   gather_rows_kernel    rows of x by a token table (bf16; the expert-parallel send rows)
 //   quant_act_kernel      1x128 e4m3 activation quantisation
-//   gather_fp8_kernel     x_q / scales gathered into expert order
+//   quant_scatter_fp8_kernel  the quantisation and the copy into expert order, token-major
 //   moe_gemm_kernel       tcgen05 grouped GEMM, one CTA per tile (moe_gemm.cuh)
 //   moe_gemm_fp8_kernel   the same for e4m3 with block scales (moe_gemm_fp8.cuh)
 //   moe_gemm2_kernel      CTA-pair grouped GEMM, cta_group::2 (moe_gemm2.cuh)
@@ -554,6 +555,21 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(const void* __restric
 // One warp per (token, 128-channel block), 4 channels per lane:
 //   sx = amax / 448 (1 when the block is all zero), q = e4m3_rn_sat(x / sx),
 // with the divides correctly rounded in fp32, so the codes are reproducible.
+// One lane's four consecutive channels of a 1x128 block held by the warp:
+// sx = amax / 448 over the block (1 when it is all zero), codes e4m3_rn_sat(x / sx)
+// with correctly rounded divides.  Returns the four codes (channel 0 in the low
+// byte) and the block's scale.
+__device__ __forceinline__ uint32_t quant_block_lane4(float x0, float x1, float x2, float x3, float* scale_out) {
+    float amax = fmaxf(fmaxf(fabsf(x0), fabsf(x1)), fmaxf(fabsf(x2), fabsf(x3)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    *scale_out = scale;
+    const uint32_t lo = cvt_e4m3x2(__fdiv_rn(x1, scale), __fdiv_rn(x0, scale));
+    const uint32_t hi = cvt_e4m3x2(__fdiv_rn(x3, scale), __fdiv_rn(x2, scale));
+    return lo | (hi << 16);
+}
+
 __global__ void __launch_bounds__(256) quant_act_kernel(const __nv_bfloat16* __restrict__ x, int T, int d,
                                                         uint8_t* __restrict__ q, float* __restrict__ sx) {
     const int nb = d / 128;
@@ -565,31 +581,53 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const __nv_bfloat16* __r
     const uint2 raw = *reinterpret_cast<const uint2*>(x + off);
     const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
     const float2 a = __bfloat1622float2(p2[0]), c = __bfloat1622float2(p2[1]);
-    float amax = fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(c.x), fabsf(c.y)));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-    const uint32_t lo = cvt_e4m3x2(__fdiv_rn(a.y, scale), __fdiv_rn(a.x, scale));
-    const uint32_t hi = cvt_e4m3x2(__fdiv_rn(c.y, scale), __fdiv_rn(c.x, scale));
-    *reinterpret_cast<uint32_t*>(q + off) = lo | (hi << 16);
+    float scale;
+    *reinterpret_cast<uint32_t*>(q + off) = quant_block_lane4(a.x, a.y, c.x, c.y, &scale);
     if (lane == 0) sx[(size_t)t * nb + b] = scale;
 }
 
-__global__ void __launch_bounds__(256) gather_fp8_kernel(const uint8_t* __restrict__ xq, const float* __restrict__ sx,
-                                                         int d, int n_tok, const int32_t* __restrict__ row_tok,
-                                                         const int32_t* __restrict__ n_rows_dev, int rows_ld,
-                                                         uint8_t* __restrict__ xpq, float* __restrict__ sxT) {
-    int n_rows = *n_rows_dev;
-    // checking build: the row count fits the permuted buffers, every row's token exists
-    if (kDebugChecks && !dbg_ok(n_rows >= 0 && n_rows <= rows_ld)) n_rows = n_rows < 0 ? 0 : rows_ld;
-    const int nvec = d / 16, nb = d / 128;
-    for (int r = blockIdx.x; r < n_rows; r += gridDim.x) {
-        const int t = row_tok[r];
-        if (kDebugChecks && !dbg_ok((unsigned)t < (unsigned)n_tok)) continue;  // uniform over the block
-        const uint4* src = reinterpret_cast<const uint4*>(xq + (size_t)t * d);
-        uint4* dst = reinterpret_cast<uint4*>(xpq + (size_t)r * d);
-        for (int v = threadIdx.x; v < nvec; v += blockDim.x) dst[v] = src[v];
-        for (int b = threadIdx.x; b < nb; b += blockDim.x) sxT[(size_t)b * rows_ld + r] = sx[(size_t)t * nb + b];
+// S6 and the copy into expert order in one token-major pass: a CTA takes token t,
+// its warps quantise the row's 1x128 blocks (quant_block_lane4, the arithmetic of
+// quant_act_kernel) and write codes and scale to every permuted row of the token:
+// inv[t*k + j] >= 0 and, when shared_base_dev is set, *shared_base_dev + t.  With
+// xq_in set (codes made by the pre-norm) the codes and scales are copied instead.
+// Codes [rows, d]; scales K-block major, sxT[b * rows_ld + row].
+__global__ void __launch_bounds__(256) quant_scatter_fp8_kernel(
+    const __nv_bfloat16* __restrict__ x, const uint8_t* __restrict__ xq_in, const float* __restrict__ sx_in, int d,
+    int T, int k, const int32_t* __restrict__ inv, const int32_t* __restrict__ shared_base_dev, int rows_ld,
+    uint8_t* __restrict__ xpq, float* __restrict__ sxT) {
+    __shared__ int s_rows[33];  // top_k <= 32, + the shared-expert row
+    const int nb = d / 128, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int shared_base = shared_base_dev ? *shared_base_dev : -1;
+    for (int t = blockIdx.x; t < T; t += gridDim.x) {
+        __syncthreads();  // the previous token's rows are no longer read
+        if (threadIdx.x <= k) {
+            int row = threadIdx.x < k ? inv[(size_t)t * k + threadIdx.x] : (shared_base >= 0 ? shared_base + t : -1);
+            // checking build: a row inside the permuted buffers (else it is skipped)
+            if (kDebugChecks && row >= 0 && !dbg_ok(row < rows_ld)) row = -1;
+            s_rows[threadIdx.x] = row;
+        }
+        __syncthreads();
+        for (int b = warp; b < nb; b += blockDim.x / 32) {
+            const size_t off = (size_t)t * d + (size_t)b * 128 + lane * 4;
+            uint32_t code;
+            float scale;
+            if (xq_in) {
+                code = *reinterpret_cast<const uint32_t*>(xq_in + off);
+                scale = sx_in[(size_t)t * nb + b];
+            } else {
+                const uint2 raw = *reinterpret_cast<const uint2*>(x + off);
+                const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+                const float2 a = __bfloat1622float2(p2[0]), c = __bfloat1622float2(p2[1]);
+                code = quant_block_lane4(a.x, a.y, c.x, c.y, &scale);
+            }
+            for (int jr = 0; jr <= k; ++jr) {
+                const int row = s_rows[jr];
+                if (row < 0) continue;  // uniform over the block
+                *reinterpret_cast<uint32_t*>(xpq + (size_t)row * d + (size_t)b * 128 + lane * 4) = code;
+                if (lane == 0) sxT[(size_t)b * rows_ld + row] = scale;
+            }
+        }
     }
 }
 
@@ -1096,16 +1134,6 @@ cudaError_t launch_quant_act(const __nv_bfloat16* x, int T, int d, uint8_t* q, f
     return cudaGetLastError();
 }
 
-cudaError_t launch_gather_fp8(const uint8_t* xq, const float* sx, int d, int n_tok, const int32_t* row_tok,
-                              const int32_t* n_rows_dev, int max_rows, uint8_t* xpq, float* sxT, int n_sm,
-                              cudaStream_t s) {
-    int grid = max_rows < n_sm * 8 ? max_rows : n_sm * 8;
-    if (grid < 1) grid = 1;
-    note_launch();
-    gather_fp8_kernel<<<grid, 256, 0, s>>>(xq, sx, d, n_tok, row_tok, n_rows_dev, max_rows, xpq, sxT);
-    return cudaGetLastError();
-}
-
 cudaError_t launch_router_f32(const float* x, const __nv_bfloat16* wr, int T, int d, int E, float* logits,
                               cudaStream_t s) {
     note_launch();
@@ -1185,6 +1213,16 @@ cudaError_t launch_gather(const void* x, bool x_f32, int d, int n_tok, const int
     if (grid < 1) grid = 1;
     note_launch();
     gather_rows_kernel<<<grid, 256, 0, s>>>(x, x_f32 ? 1 : 0, d, n_tok, row_tok, n_rows_dev, max_rows, x_perm);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_scatter_fp8(const __nv_bfloat16* x, const uint8_t* xq_in, const float* sx_in, int d, int T,
+                                     int k, const int32_t* inv, const int32_t* shared_base_dev, int rows_ld,
+                                     uint8_t* xpq, float* sxT, int n_sm, cudaStream_t s) {
+    int grid = T < n_sm * 8 ? T : n_sm * 8;
+    if (grid < 1) grid = 1;
+    note_launch();
+    quant_scatter_fp8_kernel<<<grid, 256, 0, s>>>(x, xq_in, sx_in, d, T, k, inv, shared_base_dev, rows_ld, xpq, sxT);
     return cudaGetLastError();
 }
 

@@ -120,10 +120,10 @@ cudaError_t launch_scatter_rows(const void* x, bool x_f32, int d, int T, int k, 
                                 cudaStream_t s);
 // q[t, :], sx[t, b]: per-token, per-128-channel e4m3 quantisation of bf16 x
 cudaError_t launch_quant_act(const __nv_bfloat16* x, int T, int d, uint8_t* q, float* sx, cudaStream_t s);
-// xpq[r, :] = xq[row_tok[r], :]; sxT[b][r] = sx[row_tok[r], b] for r < row_off[n_groups]
-cudaError_t launch_gather_fp8(const uint8_t* xq, const float* sx, int d, int n_tok, const int32_t* row_tok,
-                              const int32_t* n_rows_dev, int max_rows, uint8_t* xpq, float* sxT, int n_sm,
-                              cudaStream_t s);
+// S6 + copy into expert order, token-major (xq_in set: copy codes and scales made earlier)
+cudaError_t launch_quant_scatter_fp8(const __nv_bfloat16* x, const uint8_t* xq_in, const float* sx_in, int d, int T,
+                                     int k, const int32_t* inv, const int32_t* shared_base_dev, int rows_ld,
+                                     uint8_t* xpq, float* sxT, int n_sm, cudaStream_t s);
 // checking build, tests only: *p = v on the stream
 cudaError_t launch_debug_poke(int32_t* p, int v, cudaStream_t s);
 int gemm_fp8_smem_bytes(int mode, int bn);
