@@ -41,10 +41,16 @@ def run(W, x, y_dtype, accumulate=False, y0=None):
     ws = torch.empty(moe.dense_workspace_size(d, hidden, act, moe.MOE_E4M3 if fp8 else moe.MOE_BF16, T),
                      dtype=torch.uint8, device=DEV)
     y = y0.clone() if y0 is not None else torch.empty((T, d), dtype=y_dtype, device=DEV)
+    n0 = moe.launch_count()
     moe.moe_dense_ffn(W["w_gate"], W["w_up"], W["w_down"], x, y, W.get("s_gate"), W.get("s_up"), W.get("s_down"),
                       accumulate=accumulate, workspace=ws)
+    n = moe.launch_count() - n0
     torch.cuda.synchronize()
     assert moe.device_error() == 0
+    # the tables, a copy of x into row order only for fp32 x (the bf16 cast) or e4m3 weights (the
+    # quantisation), the two GEMMs, the bf16 cast of y
+    copy = 1 if (fp8 or x.dtype == torch.float32) else 0
+    assert n == 1 + copy + 2 + (1 if y.dtype == torch.bfloat16 else 0)
     return y
 
 
