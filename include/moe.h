@@ -470,11 +470,12 @@ MOE_API int moe_abi_version(void);
 /* ---- Checking build ------------------------------------------------------
  * The library also comes as libmoe_b200_debug.so, the same sources compiled
  * with MOE_DEBUG.  Its kernels check, before every access that depends on a
- * device-built table, that the access stays inside its buffer: the token of
- * each permuted row (x rows when gathering, y rows in the combine), the row
- * count and the row range of every grouped-GEMM work item against the
- * permuted buffers, and each item's weight tile against the expert's weight
- * matrix (so every TMA coordinate lies inside its tensor map).  A failed
+ * device-built table, that the access stays inside its buffer: the permuted
+ * row each token is copied to, the token of each row the combine adds into
+ * y, the row count and the row range of every grouped-GEMM work item against
+ * the permuted buffers and against the group's item count, and each item's
+ * weight tile against the expert's weight matrix (so every TMA coordinate
+ * lies inside its tensor map).  A failed
  * check sets MOE_DEVERR_BOUNDS and skips the access, or replaces the work
  * item with an in-bounds one whose output is discarded as wrong; nothing
  * traps.  It stands in for a memory checker, at the cost of a few
