@@ -1,5 +1,5 @@
 """Layer configurations beyond the five workloads, checked in full against the oracle:
-no shared expert, other expert / group / top-k counts, a shared expert wider than the
+no shared expert (bf16 x, fp32 x, e4m3 weights), other expert / group / top-k counts, a shared expert wider than the
 routed ones, no group limiting (one group), and every token routed to the same eight
 experts (the largest per-expert row count, T rows each, on the CTA-pair kernels)."""
 import dataclasses
@@ -25,6 +25,11 @@ CASES = {
     "one_group_k1": (dict(n_experts=32, n_groups=1, topk_groups=1, top_k=1, x_f32=False), 1),
     "fp8_e32": (dict(d=512, n_experts=32, n_groups=4, topk_groups=2, top_k=4, hidden=256, shared_hidden=256,
                      x_f32=False, fp8=True), 1),
+    # no shared row in the copy into expert order: fp32 x (converted in the copy) and e4m3 weights
+    # (quantised in the copy)
+    "no_shared_f32": (dict(x_f32=True), 0),
+    "fp8_e32_no_shared": (dict(d=512, n_experts=32, n_groups=4, topk_groups=2, top_k=4, hidden=256,
+                               shared_hidden=256, x_f32=False, fp8=True), 0),
 }
 
 
