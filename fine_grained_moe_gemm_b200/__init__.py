@@ -121,6 +121,10 @@ def _configure(L):
     L.moe_ep_dispatch_packed.argtypes = [ctypes.POINTER(MoeConfig), I, I, P, P, P, I, P, P, P, P]
     L.moe_ep_unpack.restype = I
     L.moe_ep_unpack.argtypes = [ctypes.POINTER(MoeConfig), I, P, P, P, P, P]
+    L.moe_ep_dispatch_peer.restype = I
+    L.moe_ep_dispatch_peer.argtypes = [ctypes.POINTER(MoeConfig), I, I, I, P, P, P, I, P, P, P, P]
+    L.moe_ep_combine_peer.restype = I
+    L.moe_ep_combine_peer.argtypes = [I, I, I, I, I, P, P, P, P, P, P]
     L.moe_forward_noalloc.restype = I
     L.moe_forward_noalloc.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, I, P, I, I, P]
     L.moe_debug_build.restype = I
@@ -430,6 +434,55 @@ def moe_ep_dispatch_packed(cfg: MoeConfig, n_ranks: int, capacity: int, topk_idx
     _check(lib().moe_ep_dispatch_packed(ctypes.byref(cfg), int(n_ranks), int(capacity), _p(topk_idx), _p(topk_w),
                                         _p(x), T, _p(send_counts), _p(send_tok), _p(packed), _stream(stream)),
            "moe_ep_dispatch_packed")
+
+
+def _ptr_array(ptrs, n: int, name: str):
+    """A device array of n device pointers: an int64 CUDA tensor of n entries, or the raw address of one."""
+    if isinstance(ptrs, torch.Tensor):
+        _dev(ptrs, name)
+        if ptrs.dtype != torch.int64 or ptrs.numel() != n or not ptrs.is_contiguous():
+            raise ValueError(f"{name}: expected {n} contiguous int64 device pointers, got {tuple(ptrs.shape)} "
+                             f"{ptrs.dtype}")
+        return _p(ptrs)
+    return ctypes.c_void_p(int(ptrs))
+
+
+def moe_ep_dispatch_peer(cfg: MoeConfig, n_ranks: int, capacity: int, my_rank: int, topk_idx, topk_w, x,
+                         send_counts, send_tok, recv_bufs, stream=None):
+    """Peer-memory packed dispatch: rank q's rows written straight into rank q's receive buffer (entry q of
+    ``recv_bufs``, n_ranks device pointers) at slots [my_rank*capacity, ...), padding marked as in
+    moe_ep_dispatch_packed; ``send_tok`` [n_ranks*capacity] as there."""
+    T = x.shape[0]
+    for n, t in (("topk_idx", topk_idx), ("topk_w", topk_w), ("x", x), ("send_counts", send_counts),
+                 ("send_tok", send_tok)):
+        _dev(t, n)
+    k, slots = cfg.top_k, n_ranks * capacity
+    _shape(topk_idx, "topk_idx", (T, k), (torch.int32,))
+    _shape(topk_w, "topk_w", (T, k), (torch.float32,))
+    _shape(x, "x", (T, cfg.d), _ACT.get(cfg.act_dtype, ()))
+    _shape(send_counts, "send_counts", (n_ranks,), (torch.int32,))
+    _shape(send_tok, "send_tok", (slots,), (torch.int32,))
+    _check(lib().moe_ep_dispatch_peer(ctypes.byref(cfg), int(n_ranks), int(capacity), int(my_rank), _p(topk_idx),
+                                      _p(topk_w), _p(x), T, _p(send_counts), _p(send_tok),
+                                      _ptr_array(recv_bufs, n_ranks, "recv_bufs"), _stream(stream)),
+           "moe_ep_dispatch_peer")
+
+
+def moe_ep_combine_peer(n_ranks: int, capacity: int, my_rank: int, result_bufs, send_tok, y_acc, y=None,
+                        residual=None, stream=None):
+    """Peer-memory combine: this rank's slot i read from the result buffer of rank i // capacity (entry of
+    ``result_bufs``, n_ranks device pointers to [n_ranks*capacity, d] fp32) at row my_rank*capacity +
+    i % capacity and added into y_acc[send_tok[i]]; then y = bf16(y_acc + residual) when ``y`` is given."""
+    for n, t in (("send_tok", send_tok), ("y_acc", y_acc), ("y", y), ("residual", residual)):
+        _dev(t, n)
+    T, d = y_acc.shape
+    _shape(y_acc, "y_acc", (T, d), (torch.float32,))
+    _shape(send_tok, "send_tok", (n_ranks * capacity,), (torch.int32,))
+    _shape(y, "y", (T, d), (torch.bfloat16,))
+    _shape(residual, "residual", (T, d), (torch.bfloat16,))
+    _check(lib().moe_ep_combine_peer(T, d, int(n_ranks), int(capacity), int(my_rank),
+                                     _ptr_array(result_bufs, n_ranks, "result_bufs"), _p(send_tok), _p(y_acc), _p(y),
+                                     _p(residual), _stream(stream)), "moe_ep_combine_peer")
 
 
 def moe_ep_unpack(cfg: MoeConfig, packed, x_rows, topk_idx, topk_w, stream=None):

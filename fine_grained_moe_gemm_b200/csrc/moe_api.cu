@@ -733,6 +733,26 @@ moe_status moe_ep_dispatch_packed(const moe_config* cfg, int n_ranks, int capaci
                                                  (cudaStream_t)stream));
 }
 
+moe_status moe_ep_dispatch_peer(const moe_config* cfg, int n_ranks, int capacity, int my_rank, const int32_t* topk_idx,
+                                const float* topk_w, const void* x, int T, int32_t* send_counts, int32_t* send_tok,
+                                void* const* recv_bufs, moe_stream_t stream) {
+    NvtxRange nvtx_call("moe_ep_dispatch_peer");
+    moe_status st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (T < 0 || capacity < T || capacity < 1 || n_ranks < 1 || n_ranks > 32 || cfg->n_experts % n_ranks != 0 ||
+        my_rank < 0 || my_rank >= n_ranks || (long long)n_ranks * capacity > INT32_MAX)
+        return MOE_ERR_INVALID_ARG;
+    if (!send_counts || !send_tok || !recv_bufs || (reinterpret_cast<uintptr_t>(recv_bufs) & 7u))
+        return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!topk_idx || !topk_w || !x || !aligned16(x))) return MOE_ERR_INVALID_ARG;
+    DevInfo di;
+    if ((st = check_device(&di)) != MOE_OK) return st;
+    return cuda_status(launch_ep_dispatch_packed(
+        topk_idx, topk_w, T, cfg->top_k, cfg->n_experts, n_ranks, capacity, x, cfg->act_dtype == MOE_F32, cfg->d,
+        send_counts, send_tok, nullptr, (int)moe_ep_packed_row_bytes(cfg), (cudaStream_t)stream,
+        reinterpret_cast<uint8_t* const*>(recv_bufs), my_rank * capacity));
+}
+
 moe_status moe_ep_unpack(const moe_config* cfg, int n_rows, const void* packed, void* x_rows, int32_t* topk_idx,
                          float* topk_w, moe_stream_t stream) {
     moe_status st = check_config(cfg);
@@ -817,6 +837,29 @@ moe_status moe_ep_combine(int T, int d, int n_rows, const float* back_rows, cons
     if (st != MOE_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
     if (launch_ep_combine(back_rows, send_tok, n_rows, T, d, y_acc, di.sm_count, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (y && launch_finalize_bf16(y_acc, static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(y),
+                                  (size_t)T * d, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+moe_status moe_ep_combine_peer(int T, int d, int n_ranks, int capacity, int my_rank, const float* const* result_bufs,
+                               const int32_t* send_tok, float* y_acc, void* y, const void* residual,
+                               moe_stream_t stream) {
+    if (T < 0 || d <= 0 || d % 8 != 0 || n_ranks < 1 || n_ranks > 32 || capacity < 1 || capacity < T ||
+        my_rank < 0 || my_rank >= n_ranks || (long long)n_ranks * capacity > INT32_MAX)
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!y_acc || !aligned16(y_acc) || !send_tok || !result_bufs || (reinterpret_cast<uintptr_t>(result_bufs) & 7u) ||
+        (y && !aligned16(y)) || (residual && !aligned16(residual)))
+        return MOE_ERR_INVALID_ARG;
+    DevInfo di;
+    moe_status st = check_device(&di);
+    if (st != MOE_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (launch_ep_combine(nullptr, send_tok, n_ranks * capacity, T, d, y_acc, di.sm_count, s, result_bufs, capacity,
+                          my_rank * capacity) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (y && launch_finalize_bf16(y_acc, static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(y),
                                   (size_t)T * d, s) != cudaSuccess)

@@ -905,14 +905,25 @@ __global__ void __launch_bounds__(256) ep_rows_kernel(const int32_t* __restrict_
 
 // Packed dispatch rows (fixed-capacity layout): row r = bf16 x [d] | ids int32 [k] |
 // weights fp32 [k] | padding to row_bytes.  One CTA per row; a padding slot (token
-// -1) gets ids -1 (its x and weights are left as they are).
+// -1) gets ids -1 (its x and weights are left as they are).  Row r (destination rank
+// q = r / capacity, slot i = r % capacity) goes to packed + r * row_bytes, or, with
+// dst_rank set (peer form), straight into rank q's receive buffer at slot
+// dst_row0 + i: dst_rank[q] + (dst_row0 + i) * row_bytes.
 __global__ void __launch_bounds__(128) ep_pack_kernel(const int32_t* __restrict__ idx, const float* __restrict__ w,
                                                       int k, const void* __restrict__ x, int x_f32, int d,
                                                       const int32_t* __restrict__ send_tok,
-                                                      uint8_t* __restrict__ packed, int row_bytes) {
+                                                      uint8_t* __restrict__ packed, int row_bytes,
+                                                      uint8_t* const* __restrict__ dst_rank, int capacity,
+                                                      int dst_row0) {
     const int r = blockIdx.x;
     const int t = send_tok[r];
-    uint8_t* row = packed + (size_t)r * row_bytes;
+    uint8_t* row;
+    if (dst_rank) {
+        const int q = r / capacity;
+        row = dst_rank[q] + (size_t)(dst_row0 + (r - q * capacity)) * row_bytes;
+    } else {
+        row = packed + (size_t)r * row_bytes;
+    }
     int32_t* ids = reinterpret_cast<int32_t*>(row + (size_t)d * 2);
     float* ws = reinterpret_cast<float*>(row + (size_t)d * 2 + (size_t)k * 4);
     if (t < 0) {
@@ -961,10 +972,15 @@ __global__ void __launch_bounds__(128) ep_unpack_kernel(const uint8_t* __restric
     for (int v = threadIdx.x; v < d / 8; v += blockDim.x) dst[v] = src[v];
 }
 
-// combine: acc[send_tok[r], :] += back[r, :] (the partial sums the ranks returned)
+// combine: acc[send_tok[r], :] += back[r, :] (the partial sums the ranks returned),
+// or, with src_rank set (peer form), the row read straight from the result buffer of
+// the rank that computed it: src_rank[q] + (src_row0 + i) * d for q = r / capacity,
+// i = r % capacity.
 __global__ void __launch_bounds__(256) ep_combine_kernel(const float* __restrict__ back,
                                                          const int32_t* __restrict__ send_tok, int n_rows, int T,
-                                                         int d, float* __restrict__ acc) {
+                                                         int d, float* __restrict__ acc,
+                                                         const float* const* __restrict__ src_rank, int capacity,
+                                                         int src_row0) {
     const int d4 = d / 4;
     const size_t n = (size_t)n_rows * d4;
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
@@ -976,7 +992,14 @@ __global__ void __launch_bounds__(256) ep_combine_kernel(const float* __restrict
             set_dev_error(MOE_DEVERR_BAD_ROWS);
             continue;
         }
-        const float4 v = *reinterpret_cast<const float4*>(back + r * d + c);
+        const float* src;
+        if (src_rank) {
+            const int q = (int)(r / capacity);
+            src = src_rank[q] + (size_t)(src_row0 + (int)(r - (size_t)q * capacity)) * d;
+        } else {
+            src = back + r * d;
+        }
+        const float4 v = *reinterpret_cast<const float4*>(src + c);
         float* dst = acc + (size_t)t * d + c;
         atomicAdd(dst + 0, v.x);
         atomicAdd(dst + 1, v.y);
@@ -1318,14 +1341,16 @@ cudaError_t launch_ep_dispatch(const int32_t* idx, const float* w, int T, int k,
 
 cudaError_t launch_ep_dispatch_packed(const int32_t* idx, const float* w, int T, int k, int E, int R, int capacity,
                                       const void* x, bool x_f32, int d, int32_t* counts, int32_t* send_tok,
-                                      uint8_t* packed, int row_bytes, cudaStream_t s) {
+                                      uint8_t* packed, int row_bytes, cudaStream_t s, uint8_t* const* dst_rank,
+                                      int dst_row0) {
     const int epr = E / R;
     note_launch();
     ep_count_kernel<<<R, EP_THREADS, 0, s>>>(idx, T, k, E, epr, counts);
     note_launch();
     ep_place_kernel<<<R, EP_THREADS, 0, s>>>(idx, T, k, E, epr, R, counts, nullptr, send_tok, capacity);
     note_launch();
-    ep_pack_kernel<<<R * capacity, 128, 0, s>>>(idx, w, k, x, x_f32 ? 1 : 0, d, send_tok, packed, row_bytes);
+    ep_pack_kernel<<<R * capacity, 128, 0, s>>>(idx, w, k, x, x_f32 ? 1 : 0, d, send_tok, packed, row_bytes, dst_rank,
+                                                capacity, dst_row0);
     return cudaGetLastError();
 }
 
@@ -1337,13 +1362,13 @@ cudaError_t launch_ep_unpack(const uint8_t* packed, int n_rows, int row_bytes, i
 }
 
 cudaError_t launch_ep_combine(const float* back, const int32_t* send_tok, int n_rows, int T, int d, float* acc,
-                              int n_sm, cudaStream_t s) {
+                              int n_sm, cudaStream_t s, const float* const* src_rank, int capacity, int src_row0) {
     if (n_rows == 0) return cudaSuccess;
     const size_t n = (size_t)n_rows * (d / 4);
     size_t grid = (n + 255) / 256;
     if (grid > (size_t)n_sm * 16) grid = (size_t)n_sm * 16;
     note_launch();
-    ep_combine_kernel<<<(unsigned)grid, 256, 0, s>>>(back, send_tok, n_rows, T, d, acc);
+    ep_combine_kernel<<<(unsigned)grid, 256, 0, s>>>(back, send_tok, n_rows, T, d, acc, src_rank, capacity, src_row0);
     return cudaGetLastError();
 }
 

@@ -98,17 +98,22 @@ cudaError_t launch_ep_dispatch(const int32_t* idx, const float* w, int T, int k,
                                __nv_bfloat16* send_x, int32_t* send_idx, float* send_w, int n_sm, cudaStream_t s);
 // Fixed-capacity packed dispatch: rank q's rows at [q * capacity, q * capacity + counts[q]),
 // padding slots token -1 and ids -1; packed rows bf16 x | ids | weights (row_bytes each).
+// dst_rank set (peer form): the rows of rank q go to dst_rank[q] at slots dst_row0 + i
+// instead of packed (dst_rank: device array of R pointers).
 cudaError_t launch_ep_dispatch_packed(const int32_t* idx, const float* w, int T, int k, int E, int R, int capacity,
                                       const void* x, bool x_f32, int d, int32_t* counts, int32_t* send_tok,
-                                      uint8_t* packed, int row_bytes, cudaStream_t s);
+                                      uint8_t* packed, int row_bytes, cudaStream_t s,
+                                      uint8_t* const* dst_rank = nullptr, int dst_row0 = 0);
 // packed rows -> x_rows [n, d] bf16, ids [n, k], w [n, k] (padding rows: ids -1, w 0)
 cudaError_t launch_ep_unpack(const uint8_t* packed, int n_rows, int row_bytes, int d, int k, __nv_bfloat16* x_rows,
                              int32_t* ids, float* w, cudaStream_t s);
 // acc[send_tok[r], :] += back[r, :] for r < n_rows (fp32 atomics; d % 4 == 0); a token
 // of -1 is a padding slot and skipped, any other outside [0, T) sets
-// MOE_DEVERR_BAD_ROWS and its row is skipped
+// MOE_DEVERR_BAD_ROWS and its row is skipped.  src_rank set (peer form): row r read from
+// src_rank[r / capacity] at row src_row0 + r % capacity instead of back.
 cudaError_t launch_ep_combine(const float* back, const int32_t* send_tok, int n_rows, int T, int d, float* acc,
-                              int n_sm, cudaStream_t s);
+                              int n_sm, cudaStream_t s, const float* const* src_rank = nullptr, int capacity = 0,
+                              int src_row0 = 0);
 // x_perm[r, :] = x[row_tok[r], :] (fp32 input rounded to bf16) for r < row_off[n_groups]
 // (checking build: row_tok entries against n_tok, the row count against max_rows)
 cudaError_t launch_gather(const void* x, bool x_f32, int d, int n_tok, const int32_t* row_tok,

@@ -29,7 +29,15 @@ Two forms of the same layer:
                   all-to-alls have equal splits known in advance, nothing waits
                   on the host, and a forward can be captured in a CUDA graph.
                   The price is padding: each block is T_max rows whatever the
-                  count.
+                  count.  With exchange="peer" the same layer moves its rows
+                  without an all-to-all: the receive and result buffers are
+                  symmetric memory (every rank maps the others' buffers), the
+                  dispatch kernel stores each rank's packed rows straight into
+                  that rank's receive buffer and the combine kernel reads the
+                  partial sums straight from the result buffer of the rank that
+                  computed them (peer stores and loads over NVLink between GPUs);
+                  a one-element all-reduce on the stream after the dispatch and
+                  after the experts orders those accesses across the ranks.
 """
 from __future__ import annotations
 
@@ -37,8 +45,8 @@ import torch
 import torch.distributed as dist
 
 from . import (MOE_BF16, MOE_E4M3, MoeConfig, dense_workspace_size, ep_max_send_rows, ep_packed_row_bytes,
-               experts_routed_workspace_size, moe_dense_ffn, moe_ep_combine, moe_ep_dispatch, moe_ep_dispatch_packed,
-               moe_ep_unpack, moe_experts_routed, moe_route)
+               experts_routed_workspace_size, moe_dense_ffn, moe_ep_combine, moe_ep_combine_peer, moe_ep_dispatch,
+               moe_ep_dispatch_packed, moe_ep_dispatch_peer, moe_ep_unpack, moe_experts_routed, moe_route)
 
 
 def exchange_counts(send_counts: torch.Tensor, group=None) -> torch.Tensor:
@@ -125,13 +133,19 @@ class EpLayer:
     Every rank of ``group`` builds one with the same ``T_max`` and calls :meth:`forward` together.  Buffers are
     allocated here, once; a forward allocates nothing, never reads a count on the host, and its two all-to-alls
     have equal splits (T_max packed rows per peer there, T_max fp32 rows back), so on NCCL it can be captured in a
-    CUDA graph.  ``shared_hidden`` / ``shared_e4m3`` size the shared expert's workspace."""
+    CUDA graph.  ``shared_hidden`` / ``shared_e4m3`` size the shared expert's workspace.
+
+    ``exchange``: "all_to_all" (NCCL all-to-alls of the packed rows and of the partial sums) or "peer" (the
+    receive and result buffers in symmetric memory; the dispatch stores into the peers' receive buffers and the
+    combine loads from their result buffers, with an all-reduce of one element after each as the fence)."""
 
     def __init__(self, cfg: MoeConfig, T_max: int, device, group=None, shared_hidden: int | None = None,
-                 shared_e4m3: bool = False):
+                 shared_e4m3: bool = False, exchange: str = "all_to_all"):
         if cfg.n_shared != 1:
             raise ValueError("the expert-parallel layer takes one shared expert")
-        self.cfg, self.T_max, self.group = cfg, int(T_max), group
+        if exchange not in ("all_to_all", "peer"):
+            raise ValueError(f"exchange: {exchange!r}, expected 'all_to_all' or 'peer'")
+        self.cfg, self.T_max, self.group, self.exchange = cfg, int(T_max), group, exchange
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
         self.lo, self.n_local = expert_block(cfg, self.rank, self.world)
@@ -145,13 +159,17 @@ class EpLayer:
         self.w = torch.empty((self.T_max, k), dtype=f32, device=dev)
         self.counts = torch.empty(self.world, dtype=i32, device=dev)
         self.send_tok = torch.empty(slots, dtype=i32, device=dev)
-        self.send = torch.empty((slots, rb), dtype=torch.uint8, device=dev)
-        self.recv = torch.empty((slots, rb), dtype=torch.uint8, device=dev)
+        self.send = torch.empty((slots, rb), dtype=torch.uint8, device=dev) if exchange == "all_to_all" else None
+        self.recv = self._buffer((slots, rb), torch.uint8, dev)
         self.recv_x = torch.empty((slots, d), dtype=torch.bfloat16, device=dev)
         self.recv_idx = torch.empty((slots, k), dtype=i32, device=dev)
         self.recv_w = torch.empty((slots, k), dtype=f32, device=dev)
-        self.recv_y = torch.empty((slots, d), dtype=f32, device=dev)
-        self.back = torch.empty((slots, d), dtype=f32, device=dev)
+        self.recv_y = self._buffer((slots, d), f32, dev)
+        self.back = torch.empty((slots, d), dtype=f32, device=dev) if exchange == "all_to_all" else None
+        if exchange == "peer":
+            self.recv_ptrs = self._peer_pointers(self.recv)
+            self.result_ptrs = self._peer_pointers(self.recv_y)
+            self.fence_buf = torch.zeros(1, dtype=torch.int32, device=dev)
         self.y_acc = torch.empty((self.T_max, d), dtype=f32, device=dev)
         self.ws = torch.empty(max(experts_routed_workspace_size(cfg, self.n_local, slots), 1), dtype=torch.uint8,
                               device=dev)
@@ -160,6 +178,27 @@ class EpLayer:
         self.dws = torch.empty(max(dense_workspace_size(d, hs, cfg.act_dtype, wdt, self.T_max), 1),
                                dtype=torch.uint8, device=dev)
 
+    def _buffer(self, shape, dtype, dev):
+        if self.exchange == "all_to_all":
+            return torch.empty(shape, dtype=dtype, device=dev)
+        import torch.distributed._symmetric_memory as symm_mem
+        return symm_mem.empty(*shape, dtype=dtype, device=dev)
+
+    def _peer_pointers(self, buf: torch.Tensor) -> torch.Tensor:
+        """Device array of every rank's address of ``buf`` (a symmetric-memory tensor), as this process maps
+        them; entry ``rank`` is ``buf`` itself."""
+        import torch.distributed._symmetric_memory as symm_mem
+        handle = symm_mem.rendezvous(buf, self.group if self.group is not None else dist.group.WORLD)
+        ptrs = [int(p) + int(handle.offset) for p in handle.buffer_ptrs]
+        if ptrs[self.rank] != buf.data_ptr():
+            raise RuntimeError("symmetric memory: this rank's mapped address is not the tensor's")
+        self._handles = getattr(self, "_handles", []) + [handle]  # the mappings live as long as the layer
+        return torch.tensor(ptrs, dtype=torch.int64, device=buf.device)
+
+    def _fence(self):
+        """Every rank's earlier kernels on this stream are done before any rank's later ones start."""
+        dist.all_reduce(self.fence_buf, group=self.group)
+
     def forward(self, w_router, local_weights: dict, shared_weights: dict, bias, x, y, residual=None):
         """y = MoE(x) (+ residual) for this rank's tokens x [T, d], T <= T_max; arguments as moe_forward_ep."""
         cfg, T = self.cfg, x.shape[0]
@@ -167,19 +206,32 @@ class EpLayer:
             raise ValueError(f"{T} tokens, the layer was built for at most {self.T_max}")
         # (1) routing of this rank's tokens, (2) dispatch into fixed-capacity packed rows
         moe_route(cfg, x, w_router, self.logits[:T], bias, self.idx[:T], self.w[:T])
-        moe_ep_dispatch_packed(cfg, self.world, self.T_max, self.idx[:T], self.w[:T], x, self.counts, self.send_tok,
-                               self.send)
-        # (3) rows to their ranks: equal blocks of T_max rows, no counts needed
-        dist.all_to_all_single(self.recv, self.send, group=self.group)
+        if self.exchange == "peer":
+            # (2+3) the packed rows stored straight into each rank's receive buffer
+            moe_ep_dispatch_peer(cfg, self.world, self.T_max, self.rank, self.idx[:T], self.w[:T], x, self.counts,
+                                 self.send_tok, self.recv_ptrs)
+            self._fence()
+        else:
+            moe_ep_dispatch_packed(cfg, self.world, self.T_max, self.idx[:T], self.w[:T], x, self.counts,
+                                   self.send_tok, self.send)
+            # (3) rows to their ranks: equal blocks of T_max rows, no counts needed
+            dist.all_to_all_single(self.recv, self.send, group=self.group)
         # (4) this rank's experts on every received slot (padding slots carry no local expert)
         moe_ep_unpack(cfg, self.recv, self.recv_x, self.recv_idx, self.recv_w)
         moe_experts_routed(cfg, local_weights, self.lo, self.n_local, self.recv_x, self.recv_idx, self.recv_w,
                            self.recv_y, workspace=self.ws)
-        # (5) partial sums back, block for block
-        dist.all_to_all_single(self.back, self.recv_y, group=self.group)
+        # (5) partial sums back, block for block (peer: left in place, read by the combine)
+        if self.exchange == "peer":
+            self._fence()
+        else:
+            dist.all_to_all_single(self.back, self.recv_y, group=self.group)
         # (6) the shared expert on this rank's tokens, (7) combine (padding slots skipped)
         if T:
             moe_dense_ffn(shared_weights["w_gate"], shared_weights["w_up"], shared_weights["w_down"], x,
                           self.y_acc[:T], shared_weights.get("s_gate"), shared_weights.get("s_up"),
                           shared_weights.get("s_down"), workspace=self.dws)
-            moe_ep_combine(self.back, self.send_tok, self.y_acc[:T], y, residual)
+            if self.exchange == "peer":
+                moe_ep_combine_peer(self.world, self.T_max, self.rank, self.result_ptrs, self.send_tok,
+                                    self.y_acc[:T], y, residual)
+            else:
+                moe_ep_combine(self.back, self.send_tok, self.y_acc[:T], y, residual)

@@ -380,6 +380,26 @@ MOE_API moe_status moe_ep_dispatch_packed(const moe_config* cfg, int n_ranks, in
                                           const float* topk_w, const void* x, int T, int32_t* send_counts,
                                           int32_t* send_tok, void* packed, moe_stream_t stream);
 
+/* Peer-memory form of the packed dispatch: the same rows written straight into
+ * every rank's receive buffer, so that no all-to-all moves them (on NVLink the
+ * stores to a peer's buffer cross the link as the kernel runs).  recv_bufs is a
+ * device array of n_ranks device pointers, entry q the receive buffer of rank q
+ * as this process addresses it (its own buffer for q == my_rank, the peers'
+ * mapped into this process, e.g. symmetric memory); each buffer holds
+ * [n_ranks * capacity, moe_ep_packed_row_bytes(cfg)] bytes, 16-byte aligned.
+ * Rank q's rows land in recv_bufs[q] at slots [my_rank * capacity, my_rank *
+ * capacity + send_counts[q]) and the rest of those capacity slots are marked as
+ * padding: after every rank has made this call, each buffer holds what
+ * moe_ep_dispatch_packed plus an equal-split all-to-all would have delivered.
+ * Ordering the stores before any rank reads its buffer is the caller's (a
+ * collective on the stream after this call on every rank does it).
+ * send_counts, send_tok and the other arguments as moe_ep_dispatch_packed;
+ * 0 <= my_rank < n_ranks; recv_bufs 8-byte aligned. */
+MOE_API moe_status moe_ep_dispatch_peer(const moe_config* cfg, int n_ranks, int capacity, int my_rank,
+                                        const int32_t* topk_idx, const float* topk_w, const void* x, int T,
+                                        int32_t* send_counts, int32_t* send_tok, void* const* recv_bufs,
+                                        moe_stream_t stream);
+
 /* Received packed rows (n_rows of them, as moe_ep_dispatch_packed lays them
  * out) into the inputs of moe_experts_routed: x_rows [n_rows, d] bf16,
  * topk_idx / topk_w [n_rows, k].  Padding rows keep ids -1 (weights 0), which
@@ -415,6 +435,19 @@ MOE_API moe_status moe_experts_routed(const moe_config* cfg, const moe_weights* 
  * row is skipped.  d a multiple of 8; arrays 16-byte aligned. */
 MOE_API moe_status moe_ep_combine(int T, int d, int n_rows, const float* back_rows, const int32_t* send_tok,
                                   float* y_acc, void* y, const void* residual, moe_stream_t stream);
+
+/* Peer-memory form of the combine for the packed layout: the partial sums of this
+ * rank's slot i (i < n_ranks * capacity, send_tok as moe_ep_dispatch_peer wrote it)
+ * are read straight from the result buffer of the rank that computed them,
+ * result_bufs[q] + (my_rank * capacity + i % capacity) * d floats with q = i /
+ * capacity (the rows moe_experts_routed wrote there over the received buffer),
+ * so no all-to-all returns them; then as moe_ep_combine.  result_bufs: device
+ * array of n_ranks device pointers (own buffer and mapped peers'), each
+ * [n_ranks * capacity, d] fp32, 16-byte aligned; the caller orders the peers'
+ * writes before this call.  capacity >= T, 0 <= my_rank < n_ranks. */
+MOE_API moe_status moe_ep_combine_peer(int T, int d, int n_ranks, int capacity, int my_rank,
+                                       const float* const* result_bufs, const int32_t* send_tok, float* y_acc,
+                                       void* y, const void* residual, moe_stream_t stream);
 
 /* Size of the device scratch array that moe_forward_noalloc uses in place of
  * a caller-provided workspace: 32 MiB.  At the DeepSeek-V3 sizes (d = 7168,

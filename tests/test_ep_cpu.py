@@ -246,6 +246,30 @@ def test_packed_entry_arguments(L):
     assert L.moe_ep_unpack(ctypes.byref(cfg), 0, None, None, None, None, None) == moe.MOE_OK
 
 
+def test_peer_entry_arguments(L):
+    """The peer-memory dispatch and combine reject bad arguments on the host, before any device work."""
+    cfg = cfg_of(WORKLOADS["decode"])
+    P = ctypes.c_void_p
+    dp = lambda R, cap, me, T, bufs=P(64), counts=P(16): L.moe_ep_dispatch_peer(
+        ctypes.byref(cfg), R, cap, me, P(16), P(16), P(16), T, counts, P(16), bufs, None)
+    assert dp(8, 3, 0, 4) == moe.MOE_ERR_INVALID_ARG            # capacity below T
+    assert dp(8, 4, 8, 4) == moe.MOE_ERR_INVALID_ARG            # rank outside [0, n_ranks)
+    assert dp(8, 4, -1, 4) == moe.MOE_ERR_INVALID_ARG
+    assert dp(3, 4, 0, 4) == moe.MOE_ERR_INVALID_ARG            # 256 experts do not split over 3
+    assert dp(8, 4, 0, 4, bufs=None) == moe.MOE_ERR_INVALID_ARG
+    assert dp(8, 4, 0, 4, bufs=P(68)) == moe.MOE_ERR_INVALID_ARG  # the pointer array misaligned
+    assert dp(8, 4, 0, 4, counts=None) == moe.MOE_ERR_INVALID_ARG
+    cp = lambda T, d, R, cap, me, bufs=P(64), tok=P(16), acc=P(16): L.moe_ep_combine_peer(
+        T, d, R, cap, me, bufs, tok, acc, None, None, None)
+    assert cp(4, 7168, 8, 3, 0) == moe.MOE_ERR_INVALID_ARG       # capacity below T
+    assert cp(4, 7168, 8, 4, 8) == moe.MOE_ERR_INVALID_ARG       # rank outside [0, n_ranks)
+    assert cp(4, 7164, 8, 4, 0) == moe.MOE_ERR_INVALID_ARG       # d not a multiple of 8
+    assert cp(4, 7168, 8, 4, 0, bufs=None) == moe.MOE_ERR_INVALID_ARG
+    assert cp(4, 7168, 8, 4, 0, tok=None) == moe.MOE_ERR_INVALID_ARG
+    assert cp(4, 7168, 8, 4, 0, acc=P(24)) == moe.MOE_ERR_INVALID_ARG  # y_acc misaligned
+    assert cp(0, 7168, 8, 4, 0, bufs=None, tok=None, acc=None) == moe.MOE_OK  # nothing to do
+
+
 def _packed_stand_ins(ep_mod):
     """CPU stand-ins of the packed dispatch / unpack that follow the header's layout
     (bf16 x | int32 ids | fp32 weights | padding; padding slots: token -1, ids -1)."""
