@@ -52,6 +52,13 @@ NCU_TRAFFIC: dict = {
     "decode": (8_586_343_754, "ce34d1ac5c0e5f75",
                "ncu capture of the 31-weight-set decode-shaped case (profile_decode), reads scaled by the weight "
                "sets streamed, 146 / 31, writes as captured"),
+    "prefill": (16_032_950_250, "ce34d1ac5c0e5f75",
+                "ncu capture of the 33-weight-set prefill-shaped case (profile_prefill, 2,056,353,792 B), "
+                "scaled by the kernel's algorithmic bytes, 15,770,583,040 / 2,022,703,104"),
+    "fp8": (13_508_693_509, "ce34d1ac5c0e5f75",
+            "ncu capture of the 33-weight-set FP8-shaped case (profile_fp8, 1,727,560,192 B), scaled by the "
+            "kernel's algorithmic bytes, 8,904,507,392 / 1,138,753,536 (the share of weight re-reads taken as "
+            "captured)"),
 }
 
 HBM_NOMINAL_GBS = 7700.0  # B200 (HGX) HBM3e nominal bandwidth, for context beside the measured copy peak
