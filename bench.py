@@ -47,18 +47,17 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # source hash the capture was taken at, how the figure was obtained).  A figure
 # is reported only while the kernel sources still hash to the recorded value.
 NCU_TRAFFIC: dict = {
-    "profile_decode": (1_825_625_344, "ce34d1ac5c0e5f75",
+    "profile_decode": (1_825_798_912, "14a34ce9cab5563a",
                        "ncu capture of this workload's gate/up GEMM: dram__bytes_read.sum + dram__bytes_write.sum"),
-    "decode": (8_586_343_754, "ce34d1ac5c0e5f75",
+    "decode": (8_586_497_379, "14a34ce9cab5563a",
                "ncu capture of the 31-weight-set decode-shaped case (profile_decode), reads scaled by the weight "
                "sets streamed, 146 / 31, writes as captured"),
-    "prefill": (16_032_950_250, "ce34d1ac5c0e5f75",
-                "ncu capture of the 33-weight-set prefill-shaped case (profile_prefill, 2,056,353,792 B), "
+    "prefill": (15_973_627_812, "14a34ce9cab5563a",
+                "ncu capture of the 33-weight-set prefill-shaped case (profile_prefill, 2,048,745,216 B), "
                 "scaled by the kernel's algorithmic bytes, 15,770,583,040 / 2,022,703,104"),
-    "fp8": (13_508_693_509, "ce34d1ac5c0e5f75",
-            "ncu capture of the 33-weight-set FP8-shaped case (profile_fp8, 1,727,560,192 B), scaled by the "
-            "kernel's algorithmic bytes, 8,904,507,392 / 1,138,753,536 (the share of weight re-reads taken as "
-            "captured)"),
+    "fp8": (8_602_558_271, "14a34ce9cab5563a",
+            "ncu capture of the 33-weight-set FP8-shaped case (profile_fp8, 1,100,138,752 B), scaled by the "
+            "kernel's algorithmic bytes, 8,904,507,392 / 1,138,753,536"),
 }
 
 HBM_NOMINAL_GBS = 7700.0  # B200 (HGX) HBM3e nominal bandwidth, for context beside the measured copy peak

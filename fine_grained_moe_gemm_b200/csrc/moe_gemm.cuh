@@ -71,6 +71,7 @@ struct GemmCfg {
 struct Item {
     int g, m, row0, nvalid, K;
     int split, n_splits;  // K range of the item: blocks [split, split+1) * KB / n_splits
+    int nch;              // token chunks of the item's group: > 1, its weight tiles are read again
     bool shared;
 };
 
@@ -91,6 +92,7 @@ __device__ __forceinline__ Item decode_item(const GemmArgs& P, int i) {
         int c = i - it.m * nch;
         it.row0 = c * BN;
         it.nvalid = min(BN, P.n_rows_single - c * BN);
+        it.nch = nch;
         it.shared = false;
         it.K = P.K_routed;
         return it;
@@ -111,6 +113,7 @@ __device__ __forceinline__ Item decode_item(const GemmArgs& P, int i) {
     // checking build: a group that owns items has rows (else the chunk count below is 0)
     if (kDebugChecks && P.rows_cap > 0 && !dbg_ok(ng > 0)) ng = 1;
     int nch = (ng + BN - 1) / BN;
+    it.nch = nch;
     const int ms = local / nch;  // tile-major, split, then token chunk (chunks of a weight slice run together)
     it.m = ms / it.n_splits;
     it.split = ms - it.m * it.n_splits;

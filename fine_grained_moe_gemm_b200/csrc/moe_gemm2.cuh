@@ -189,12 +189,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
         if (lane == 0) {
             // ------------------------------------------------ TMA producer (both CTAs)
             const uint64_t pol_w = l2_policy_evict_first();
+            const uint64_t pol_keep = l2_policy_evict_normal();
             const uint64_t pol_x = l2_policy_evict_last();
             const uint32_t full0 = mapa_shared(smem_u32(&full[0]), 0);
             int stage = 0;
             uint32_t phase = 0;
             for (int i = cluster_id; i < total; i += n_clusters) {
                 const Item it = decode_item<PAIR_BN>(P, i);
+                // weights read by several items stay in L2 for the others; the rest stream
+                const uint64_t pw = it.nch > 1 ? pol_keep : pol_w;
                 const int KB = it.K / 64;
                 int n_mma = (it.nvalid + 31) & ~31;
                 const int nh = n_mma / 2;                          // this CTA's token rows
@@ -221,8 +224,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
                     uint8_t* sb = sa + C::A_BYTES;
                     const uint32_t fb = full0 + (uint32_t)(stage * 8);
                     if (leader) mbar_arrive_expect_tx(&full[stage], bytes);
-                    tma_load_2d_pair(sa, m0, kb * 64, r0, fb, pol_w);
-                    tma_load_2d_pair(sa + C::A_TILE, m1, kb * 64, r1, fb, pol_w);
+                    tma_load_2d_pair(sa, m0, kb * 64, r0, fb, pw);
+                    tma_load_2d_pair(sa + C::A_TILE, m1, kb * 64, r1, fb, pw);
                     for (int bx = 0; bx < nbox; ++bx)
                         tma_load_2d_pair(sb + bx * PAIR_BOX_ROWS * 128, &P.b, kb * 64, brow + bx * PAIR_BOX_ROWS, fb,
                                          pol_x);

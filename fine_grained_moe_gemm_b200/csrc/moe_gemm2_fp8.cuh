@@ -173,12 +173,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR8_THREADS, 1)
         const int role = warp == 0 ? 0 : warp - 1;  // 0 A/gate, 1 up, 2 B
         if (lane == 0 && !(MODE == GEMM_DOWN && role == 1)) {
             const uint64_t pol_w = l2_policy_evict_first();
+            const uint64_t pol_keep = l2_policy_evict_normal();
             const uint64_t pol_x = l2_policy_evict_last();
             const uint32_t full0 = mapa_shared(smem_u32(&full[0]), 0);
             int stage = 0;
             uint32_t phase = 0;
             for (int i = cluster_id; i < total; i += n_clusters) {
                 const Item it = decode_item<PAIR8_BN>(P, i);
+                // weights read by several items stay in L2 for the others; the rest stream
+                const uint64_t pw = it.nch > 1 ? pol_keep : pol_w;
                 const int KB = it.K / 128;
                 const int nh = ((it.nvalid + 31) & ~31) / 2;
                 const int nbox = (nh + PAIR_BOX_ROWS - 1) / PAIR_BOX_ROWS;
@@ -201,11 +204,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR8_THREADS, 1)
                     } else if (MODE == GEMM_GATEUP) {
                         // 64 gate rows over 64 up rows of this CTA's 64 features
                         const int r = base + it.m * 128 + (int)rank * 64;
-                        if (role == 0) tma_load_2d_pair(sa, it.shared ? &P.s0 : &P.a0, kb * 128, r, fb, pol_w);
-                        else tma_load_2d_pair(sa + 64 * 128, it.shared ? &P.s1 : &P.a1, kb * 128, r, fb, pol_w);
+                        if (role == 0) tma_load_2d_pair(sa, it.shared ? &P.s0 : &P.a0, kb * 128, r, fb, pw);
+                        else tma_load_2d_pair(sa + 64 * 128, it.shared ? &P.s1 : &P.a1, kb * 128, r, fb, pw);
                     } else {
                         tma_load_2d_pair(sa, it.shared ? &P.s0 : &P.a0, kb * 128, base + it.m * 256 + (int)rank * 128,
-                                         fb, pol_w);
+                                         fb, pw);
                     }
                     if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
                 }
