@@ -43,21 +43,23 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
-# kernel per launch, from one ncu capture, keyed by workload: (bytes, kernel
-# source hash the capture was taken at, how the figure was obtained).  A figure
-# is reported only while the kernel sources still hash to the recorded value.
+# kernel per launch, from one ncu capture of that kernel on the workload itself (one
+# pass of the two counters), keyed by workload: (bytes, kernel source hash the capture
+# was taken at, how the figure was obtained).  A figure is reported only while the
+# kernel sources still hash to the recorded value.
 NCU_TRAFFIC: dict = {
-    "profile_decode": (1_825_798_912, "14a34ce9cab5563a",
-                       "ncu capture of this workload's gate/up GEMM: dram__bytes_read.sum + dram__bytes_write.sum"),
-    "decode": (8_586_497_379, "14a34ce9cab5563a",
-               "ncu capture of the 31-weight-set decode-shaped case (profile_decode), reads scaled by the weight "
-               "sets streamed, 146 / 31, writes as captured"),
-    "prefill": (15_973_627_812, "14a34ce9cab5563a",
-                "ncu capture of the 33-weight-set prefill-shaped case (profile_prefill, 2,048,745,216 B), "
-                "scaled by the kernel's algorithmic bytes, 15,770,583,040 / 2,022,703,104"),
-    "fp8": (8_602_558_271, "14a34ce9cab5563a",
-            "ncu capture of the 33-weight-set FP8-shaped case (profile_fp8, 1,100,138,752 B), scaled by the "
-            "kernel's algorithmic bytes, 8,904,507,392 / 1,138,753,536"),
+    "decode": (8_614_379_008, "a8727961f91c46b0",
+              "ncu capture of this workload's moe_gemm_kernel<0, 32> launch: "
+              "dram__bytes_read.sum + dram__bytes_write.sum"),
+    "prefill": (16_396_188_160, "a8727961f91c46b0",
+               "ncu capture of this workload's moe_gemm2_kernel<0> launch: "
+               "dram__bytes_read.sum + dram__bytes_write.sum"),
+    "skewed": (9_949_065_216, "a8727961f91c46b0",
+              "ncu capture of this workload's moe_gemm2_kernel<0> launch: "
+              "dram__bytes_read.sum + dram__bytes_write.sum"),
+    "fp8": (9_804_744_704, "a8727961f91c46b0",
+           "ncu capture of this workload's moe_gemm2_fp8_kernel<0> launch: "
+           "dram__bytes_read.sum + dram__bytes_write.sum"),
 }
 
 HBM_NOMINAL_GBS = 7700.0  # B200 (HGX) HBM3e nominal bandwidth, for context beside the measured copy peak

@@ -939,6 +939,7 @@ moe_status run_experts(const moe_config* cfg, const moe_weights* wt, const Works
     g.item_off = W.item_gu;
     g.row_off = W.row_off;
     g.rows_cap = rows_max;
+    g.chunk_major = pair ? 1 : 0;  // the bf16 CTA-pair kernels
     g.n_groups = NG;
     g.n_routed = E;
     g.K_routed = g.K_shared = d;
@@ -989,6 +990,7 @@ moe_status run_experts(const moe_config* cfg, const moe_weights* wt, const Works
     dn.item_off = W.item_dn;
     dn.row_off = W.row_off;
     dn.rows_cap = rows_max;
+    dn.chunk_major = pair ? 1 : 0;
     dn.y_rows = T;
     dn.n_groups = NG;
     dn.n_routed = E;

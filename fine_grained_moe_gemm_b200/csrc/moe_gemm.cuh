@@ -104,6 +104,7 @@ __device__ __forceinline__ Item decode_item(const GemmArgs& P, int i) {
         else hi = mid - 1;
     }
     it.g = lo;
+    it.shared = lo >= P.n_routed;
     // k_splits > 1 (DOWN of a schedule with few tiles): each (tile, split) pair is one
     // item; the splits of a tile add their partial sums into y by the same atomics
     it.n_splits = P.k_splits > 1 ? P.k_splits : 1;
@@ -114,13 +115,22 @@ __device__ __forceinline__ Item decode_item(const GemmArgs& P, int i) {
     if (kDebugChecks && P.rows_cap > 0 && !dbg_ok(ng > 0)) ng = 1;
     int nch = (ng + BN - 1) / BN;
     it.nch = nch;
-    const int ms = local / nch;  // tile-major, split, then token chunk (chunks of a weight slice run together)
+    // item order inside the group: weight tile, split, then token chunk (the chunks of a
+    // weight slice run together), or, chunk-major, token chunk first (a chunk's tiles run
+    // together and the token rows stay in L2 while the weight tiles come around again)
+    int c, ms;
+    if (P.chunk_major) {
+        const int nms = (it.shared ? P.mt_shared : P.mt_routed) * it.n_splits;
+        c = local / nms;
+        ms = local - c * nms;
+    } else {
+        ms = local / nch;
+        c = local - ms * nch;
+    }
     it.m = ms / it.n_splits;
     it.split = ms - it.m * it.n_splits;
-    int c = local - ms * nch;
     it.row0 = r0 + c * BN;
     it.nvalid = min(BN, ng - c * BN);
-    it.shared = lo >= P.n_routed;
     it.K = it.shared ? P.K_shared : P.K_routed;
     if (kDebugChecks && P.rows_cap > 0) {
         // checking build: the group's rows agree with its item count, the item's rows

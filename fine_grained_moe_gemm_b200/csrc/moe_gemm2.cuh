@@ -188,9 +188,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------ TMA producer (both CTAs)
+            // chunk-major items (see decode_item): a chunk's token rows are read by its items
+            // at about the same time (normal priority), a multi-chunk expert's weight tiles
+            // again by every chunk (evict-last); single-chunk tiles stream (evict-first)
             const uint64_t pol_w = l2_policy_evict_first();
-            const uint64_t pol_keep = l2_policy_evict_normal();
-            const uint64_t pol_x = l2_policy_evict_last();
+            const uint64_t pol_keep = l2_policy_evict_last();
+            const uint64_t pol_x = l2_policy_evict_normal();
             const uint32_t full0 = mapa_shared(smem_u32(&full[0]), 0);
             int stage = 0;
             uint32_t phase = 0;

@@ -48,6 +48,8 @@ struct GemmArgs {
     // checking build: rows of the B / h buffers (0: items are not checked) and of y
     int rows_cap;
     int y_rows;
+    // grouped items token chunk outer, weight tile inner (else weight tile outer)
+    int chunk_major;
 };
 
 enum { MODE_GATEUP = 0, MODE_DOWN = 1, MODE_LOGITS = 2 };
