@@ -167,10 +167,10 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     return p;
 }
 
-// Weight tiles that more than one work item of the CTA-pair GEMMs reads (an expert
-// with several token chunks, the shared expert): kept at normal priority so that
-// the items after the first find the tile in L2 instead of streaming it again
-// (with evict_first the later chunks re-read it from HBM).
+// Normal L2 priority, for data that several work items read close together: in the
+// FP8 CTA-pair GEMM the weight tile of an expert with several token chunks (with
+// evict_first its later chunks re-read it from HBM), in the bf16 CTA-pair GEMM the
+// token rows of a chunk, which its weight tiles' items read one after another.
 __device__ __forceinline__ uint64_t l2_policy_evict_normal() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
