@@ -202,7 +202,8 @@ def test_peer_exchange_matches_the_packed_layout(name, R, cap_extra):
         moe.moe_ep_combine(back, o["tok"], acc_ref)
         torch.cuda.synchronize()
         rms = float(acc_ref.double().pow(2).mean().sqrt())
-        assert float((acc_peer - acc_ref).abs().max()) <= 1e-6 * rms     # the same sums, atomics in another order
+        # the same sums, the atomics in another order: up to eight fp32 additions an element
+        assert float((acc_peer - acc_ref).abs().max()) <= 1e-5 * rms
         assert torch.equal(y_peer, acc_peer.to(torch.bfloat16))
     assert moe.device_error() == 0
 
